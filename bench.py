@@ -1,0 +1,413 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 W4A4 linear-layer hot path on B200.
+
+One step = on-the-fly activation quantisation (static, calibrated scale) +
+the fused block-scaled FP4 GEMM with per-module global scales, on the fused
+GDN-style input projection: A = 8192 x 5120 BF16 (0.1% outlier channels),
+W = six separately calibrated modules [2048, 2048, 4096, 4096, 48, 48]
+(N = 12384), BF16 output.  Metric: TFLOPS = 2*M*N*K / step time.
+
+Timing: W untimed warm-up steps, then exactly K timed steps bracketed by a
+barrier and a device synchronise on both sides; each step is timed with CUDA
+events on the launching stream and L2 is flushed (a 256 MB write) between
+steps, outside the events.  Multi-GPU (torchrun): every rank runs its own
+replica of the step on its own batch (weak scaling, no collective on the data
+path); the reported time is the max over ranks.
+
+``--impl reference`` times the CPU oracle instead (on the host cores, rank 0
+only), on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "fused GDN-style in-proj: A 8192x5120 bf16 (0.1% x100 channels) x 6-module NVFP4 W 12384x5120"
+METRIC = "W4A4 NVFP4 GEMM TFLOPS incl. act-quant (M=8192)"
+UNIT = "TFLOPS"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--m", type=int, default=8192)
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode GB/s sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-gemm", action="store_true",
+                    help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "ptx.cuh", "quant.cuh", "nvfp4_lib.cu"):
+        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_07_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the GEMM from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "gemm_large_gdn_in_proj_8192.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """NVML samples of the SM clock and throttle reasons during the timed region."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are best effort
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(problem, rows: int, repeats: int = 1):
+    """Time the oracle's activation quantisation + FP64 GEMM on `rows` sampled
+    rows of the workload (weights quantised once, untimed).  Returns
+    (TFLOPS, seconds per repeat, threads)."""
+    import numpy as np
+    import oracle
+
+    a32 = problem.a.float().numpy()
+    s_ga = oracle.global_scale(a32)
+    qmods = oracle.quantize_modules(problem.modules)
+    w_hat = oracle.fused_weight_hat(qmods)
+    sel = np.random.default_rng(0).choice(problem.m, rows, replace=False)
+    a_rows = np.ascontiguousarray(a32[sel])
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        qa, sfa = oracle.quantize(a_rows, s_ga)
+        a_hat = oracle.dequantize(qa, sfa, s_ga)
+        oracle.gemm(a_hat, w_hat)
+    dt = (time.perf_counter() - t0) / repeats
+    flops = 2.0 * rows * problem.n * problem.k
+    return flops / dt / 1e12, dt, oracle.num_threads()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+    import numpy as np
+    import oracle
+
+    p = synthetic.gdn_in_proj(m=args.m)
+    a32 = p.a.float().numpy()
+    s_ga = oracle.global_scale(a32)
+    qmods = oracle.quantize_modules(p.modules)
+    w_hat = oracle.fused_weight_hat(qmods)
+    rows = 8
+    rng = np.random.default_rng(0)
+
+    def step():
+        sel = rng.choice(p.m, rows, replace=False)
+        qa, sfa = oracle.quantize(np.ascontiguousarray(a32[sel]), s_ga)
+        oracle.gemm(oracle.dequantize(qa, sfa, s_ga), w_hat)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2.0 * rows * p.n * p.k / dt / 1e12
+    sample = f"{rows} random rows of A per step (all {p.n} columns, K={p.k}); weights quantised once, untimed"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " (CPU oracle, row sample)", "m": p.m, "n": p.n, "k": p.k,
+                   "segments": p.widths, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local)
+    if rank == 0:
+        nvbuild.build()
+    if world > 1:
+        dist.barrier()
+    L = nv.load()
+
+    # ---- inputs resident in HBM (weights quantised offline, untimed)
+    p = synthetic.gdn_in_proj(m=args.m)
+    a_dev = p.a.to(device)
+    fw = nv.quantize_weight([w.to(device) for w in p.modules])
+    calib = nv.quantize_act(a_dev)                     # untimed calibration run -> static scale
+    act_scale = calib.scale.clone()
+    aq = nv.quantize_act(a_dev, act_scale=act_scale)
+    c = torch.empty((p.m, p.n), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    flops = 2.0 * p.m * p.n * p.k
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev):
+        if ev is not None:
+            ev[0].record(stream)
+        nv.quantize_act(a_dev, act_scale=act_scale, out=aq)
+        if ev is not None:
+            ev[1].record(stream)
+        nv.gemm(aq, fw, out=c)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step(None)
+        flush.zero_()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            step(events[i])
+            flush.zero_()
+        torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    step_ms = [e[0].elapsed_time(e[2]) for e in events]
+    gemm_ms = [e[1].elapsed_time(e[2]) for e in events]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in events]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks, peak_kind = measured_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]              # dense FP4 = 4 x dense BF16 (nominal ratio)
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak, "traffic": profiled_traffic(),
+                "kernel": "gemm_large_kernel",
+                "peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/BF16 nominal)",
+                "datasheet_fp4_frac": achieved / 9000.0}
+    quant_avg_ms = statistics.mean(quant_ms)
+    quant_bytes = p.m * p.k * 2 + p.m * p.k // 2 + p.m * p.k // 16
+    extra = {"act_quant": {"ms": quant_avg_ms, "GB/s": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
+                           "frac_hbm": quant_bytes / (quant_avg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+             "gemm_ms": gemm_avg_ms}
+
+    result = {}
+    if not args.profile_gemm:
+        result = extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, nv, synthetic, peaks)
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3, fp32 accumulate), bf16 in/out",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": p.m, "n": p.n, "k": p.k, "segments": p.widths,
+                       "act_scale": "static (calibrated)", "global_batch": p.m * world,
+                       "parallelism": f"replicas x{world}", "l2": "flushed between timed steps (256 MB write)"},
+            "roofline": roofline,
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks.summary(),
+            **extra,
+            **result,
+        }
+        if not args.profile_gemm and not args.no_cpu_baseline:
+            tf, dt, threads = time_oracle(p, rows=16, repeats=1)
+            line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                    "sample": f"16 rows of A x all {p.n} columns (activation quantisation + "
+                                              f"FP64 GEMM), {dt:.2f} s; weights quantised once, untimed"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, nv, synthetic, peaks):
+    import torch
+    out = {}
+    # ---- end to end through the public API: pinned host A in, host C out
+    a_host = p.a.pin_memory()
+    c_host = torch.empty((p.m, p.n), dtype=torch.bfloat16).pin_memory()
+    a_buf = torch.empty_like(a_dev)
+    aq = nv.quantize_act(a_dev, act_scale=act_scale)
+
+    def e2e_step():
+        a_buf.copy_(a_host, non_blocking=True)
+        nv.quantize_act(a_buf, act_scale=act_scale, out=aq)
+        nv.gemm(aq, fw, out=c)
+        c_host.copy_(c, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    n_e2e = max(3, min(args.steps, 10))
+    torch.cuda.synchronize(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = t0.elapsed_time(t1) / n_e2e
+    out["e2e"] = {"value": 2.0 * p.m * p.n * p.k / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                  "h2d_bytes_per_step": a_host.numel() * a_host.element_size(),
+                  "d2h_bytes_per_step": c_host.numel() * c_host.element_size(), "ms_per_step": e2e_ms}
+
+    # ---- dynamic activation scale (amax pass + quantise) for reference
+    ws = nv.quant_workspace(device)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(3):
+        nv.quantize_act(a_dev, workspace=ws, out=aq)
+    flush.zero_()
+    evs[0].record(stream)
+    nv.quantize_act(a_dev, workspace=ws, out=aq)
+    nv.gemm(aq, fw, out=c)
+    evs[1].record(stream)
+    torch.cuda.synchronize(device)
+    dyn_ms = evs[0].elapsed_time(evs[1])
+    out["dynamic_act_scale"] = {"value": 2.0 * p.m * p.n * p.k / (dyn_ms * 1e-3) / 1e12, "unit": UNIT,
+                                "ms_per_step": dyn_ms}
+
+    # ---- decode sweep: HBM GB/s of the small-M GEMM (L2 flushed before each launch)
+    if not args.no_decode:
+        dec = {}
+        for shape in synthetic.DECODE_SHAPES:
+            widths, k, stds = synthetic.DECODE_SHAPES[shape]
+            mods = [synthetic.weights(n_i, k, s_i, seed=1 + i).to(device) for i, (n_i, s_i) in
+                    enumerate(zip(widths, stds))]
+            fwd = nv.quantize_weight(mods)
+            del mods
+            for m in synthetic.DECODE_M:
+                a, _ = synthetic.activations(m, k, seed=0, n_outliers=0)
+                a = a.to(device)
+                aqd = nv.quantize_act(a, act_scale=act_scale)
+                cd = torch.empty((m, fwd.n), dtype=torch.bfloat16, device=device)
+                times = []
+                for it in range(13):
+                    flush.zero_()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    nv.gemm(aqd, fwd, out=cd)
+                    e1.record(stream)
+                    torch.cuda.synchronize(device)
+                    if it >= 3:
+                        times.append(e0.elapsed_time(e1))
+                ms = statistics.median(times)
+                nbytes = fwd.n * k // 2 + fwd.n * k // 16 + m * k // 2 + m * k // 16 + m * fwd.n * 2
+                gbs = nbytes / (ms * 1e-3) / 1e9
+                dec[f"m{m}_{shape}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                                        "frac_8TBs": gbs / 8000.0}
+            del fwd
+        out["decode"] = {"unit": "GB/s", "bytes": "W_q + W_sf + A_q + A_sf + C (bf16), L2 flushed",
+                         "shapes": dec}
+    return out
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,210 @@
+/*
+ * nvfp4.h - C ABI of libnvfp4: NVFP4 W4A4 linear layers on B200 (sm_100a).
+ *
+ * The method ("Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for
+ * the Recurrent Half of a Hybrid 27B LLM"):
+ *   - page summary, "Background", item 1: NVFP4 = E2M1 4-bit values, one E4M3
+ *     scale per 16-element block set to blockmax/6, one FP32 scale per tensor,
+ *     enabling native 4-bit tensor-core GEMMs;
+ *   - abstract and news article: W4A4, i.e. weights quantised once after
+ *     calibration, activations quantised on the fly;
+ *   - abstract, last sentence, and the news article's "Risks and caveats":
+ *     checkpoints calibrated per module carry one FP32 global scale per module;
+ *     when several modules are served as one fused GEMM each module's scale
+ *     must govern its own output columns (the "global-scale mismatch" fix).
+ *
+ * Conventions shared by every call:
+ *   - Pointers marked "device" are CUDA device (or managed) memory owned by the
+ *     caller; "host" pointers are ordinary host memory.  The library never
+ *     allocates or frees memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued on it and the call returns without waiting, except where a call
+ *     says it synchronises.
+ *   - Argument errors are detected before anything is enqueued and returned as
+ *     a status; nvfp4_get_last_error_string() then describes the problem.  A
+ *     failed launch returns NVFP4_ERR_CUDA.  Faults inside a kernel surface at
+ *     the caller's next synchronisation, as usual for CUDA.
+ *   - Every wait inside the kernels is bounded; a wait that runs out records a
+ *     flag that nvfp4_check_device_status() reports as NVFP4_ERR_TIMEOUT.
+ *
+ * Data layout (all row-major, "K" = reduction dimension, K % 32 == 0):
+ *   q   : rows x K/2 bytes; byte j of a row holds element 2j in its low nibble
+ *         and element 2j+1 in its high nibble; E2M1 codes 0..7 are
+ *         0, 0.5, 1, 1.5, 2, 3, 4, 6 and bit 3 is the sign.
+ *   sf  : nvfp4_sf_bytes(rows, K) bytes of UE4M3 block scales in the tiled
+ *         layout read by block-scaled tensor-core MMAs (see nvfp4_sf_offset);
+ *         padding bytes are zero.
+ *   global scale: FP32 *decode* scale s_g = amax / 2688 (2688 = 6 * 448), or
+ *         1 when that quotient is 0.  A value is x ~= e2m1 * e4m3(sb) * s_g.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad segment table, ... */
+    NVFP4_ERR_UNSUPPORTED = 2, /* a shape or mode this build does not handle */
+    NVFP4_ERR_ALIGNMENT = 3,   /* a pointer or leading dimension is not 16-byte aligned */
+    NVFP4_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out */
+    NVFP4_ERR_WORKSPACE = 6    /* workspace missing or too small */
+} nvfp4_status;
+
+typedef enum { NVFP4_IN_BF16 = 0, NVFP4_IN_FP32 = 1 } nvfp4_in_dtype;
+typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_FP32 = 1 } nvfp4_out_dtype;
+
+/* One module of a fused weight: output columns [col_begin, col_end) and that
+ * module's FP32 global (decode) scale, as returned by nvfp4_quantize_weight. */
+typedef struct {
+    int64_t col_begin;
+    int64_t col_end;
+    float w_global_scale;
+} nvfp4_segment;
+
+#define NVFP4_MAX_SEGMENTS 16
+
+/* nvfp4_gemm flags */
+#define NVFP4_GEMM_AUTO 0u          /* decode kernel for m <= 64, large kernel otherwise */
+#define NVFP4_GEMM_FORCE_LARGE 1u   /* always the persistent large-M kernel */
+#define NVFP4_GEMM_FORCE_DECODE 2u  /* always the split-K decode kernel (m <= 64) */
+
+/* ------------------------------------------------------------------------
+ * Layout helpers (pure host functions, no CUDA calls).
+ * ---------------------------------------------------------------------- */
+
+/* Bytes of a tiled scale buffer for `rows` x `k` values: rows rounded up to
+ * 128, k/16 rounded up to 4.  Returns 0 if rows < 0 or k is not a positive
+ * multiple of 16. */
+NVFP4_API size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
+
+/* Byte offset of the scale of (row, kblock) in the tiled layout, where kblock
+ * indexes 16-element blocks along K.  Scales are grouped in 512-byte atoms of
+ * 128 rows x 4 kblocks; atoms are ordered kblock-atom fastest, then 128-row
+ * block.  Inside an atom: (row % 32) * 16 + ((row % 128) / 32) * 4 +
+ * kblock % 4.  Returns -1 for out-of-range arguments. */
+NVFP4_API int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k);
+
+/* Workspace bytes nvfp4_quantize_act / nvfp4_quantize_weight need when they
+ * compute the global scale themselves (an amax accumulator). */
+NVFP4_API size_t nvfp4_quant_workspace_size(void);
+
+/* Workspace bytes nvfp4_gemm needs (currently 0 for every shape: the split-K
+ * reduction runs through distributed shared memory). */
+NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_quantize_weight - offline, per module (post-training, calibration
+ * only).  Quantises one module's n x k weight (nn.Linear layout, K
+ * contiguous, row stride ldw elements) into rows [row_offset, row_offset + n)
+ * of a fused buffer of n_total rows, so that several separately calibrated
+ * modules can be concatenated along the output dimension.
+ *
+ *   w                 device, n x k, BF16 or FP32 (dt); 16-byte aligned,
+ *                     ldw * element size a multiple of 16.
+ *   global_scale_in   host; the module's decode scale to use, or NULL to
+ *                     compute amax/2688 on the device.  Must be positive and
+ *                     finite when given.
+ *   w_q               device, n_total x k/2 bytes (this call writes its rows).
+ *   w_sf              device, nvfp4_sf_bytes(n_total, k) bytes.  This call
+ *                     writes the scale entries of its rows; the call whose
+ *                     rows end at n_total also zeroes the padding rows.
+ *   global_scale_out  host; receives the scale used (required when
+ *                     global_scale_in is NULL, may be NULL otherwise).
+ *   workspace         device, >= nvfp4_quant_workspace_size() bytes, needed
+ *                     only when global_scale_in is NULL.
+ * When the scale is computed the call SYNCHRONISES the stream to return it on
+ * the host (an offline call).
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_in_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                                   int64_t row_offset, int64_t n_total, const float* global_scale_in,
+                                   uint8_t* w_q, uint8_t* w_sf, float* global_scale_out, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_quantize_act - on-the-fly activation quantisation (the "A4" of W4A4).
+ *
+ *   a                 device, m x k, BF16 or FP32 (dt), row stride lda
+ *                     elements; 16-byte aligned rows.
+ *   act_scale_dev     device float.  Non-NULL: static (calibrated) mode, the
+ *                     tensor's decode scale is read from it.  NULL: dynamic
+ *                     mode, amax is reduced on the device first and the scale
+ *                     amax/2688 is used.
+ *   act_scale_out_dev device float receiving the scale used; required in
+ *                     dynamic mode (nvfp4_gemm reads it), optional otherwise.
+ *   a_q               device, m x k/2 bytes.
+ *   a_sf              device, nvfp4_sf_bytes(m, k) bytes (padding zeroed).
+ *   workspace         device, >= nvfp4_quant_workspace_size() bytes in
+ *                     dynamic mode (the amax accumulator), unused otherwise.
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_quantize_act(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                const float* act_scale_dev, float* act_scale_out_dev, uint8_t* a_q, uint8_t* a_sf,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_gemm - block-scaled FP4 GEMM with the per-module scale epilogue:
+ *
+ *   C[i, j] = cvt( acc[i, j] * (s_ga * w_global_scale[seg(j)]) ),
+ *   acc[i, j] = sum_k e2m1(a)[i,k] e4m3(sfa)[i,k/16] e2m1(w)[j,k] e4m3(sfw)[j,k/16]
+ *
+ * with FP32 accumulation on the tensor cores and seg(j) the segment whose
+ * [col_begin, col_end) contains column j.
+ *
+ *   a_q, a_sf         device, from nvfp4_quantize_act (m rows).
+ *   act_scale_dev     device float, s_ga (the scale nvfp4_quantize_act used).
+ *   w_q, w_sf         device, fused weight from nvfp4_quantize_weight (n rows).
+ *   segs, nsegs       host, 1..NVFP4_MAX_SEGMENTS segments, sorted, contiguous,
+ *                     first col_begin 0, last col_end n, every boundary a
+ *                     multiple of 16, scales positive and finite.
+ *   c, odt, ldc       device output, m x n, BF16 or FP32, row stride ldc
+ *                     elements (ldc >= n, 16-byte aligned rows).
+ *   workspace         device, >= nvfp4_gemm_workspace_size(...) bytes (may be
+ *                     NULL when that is 0).
+ *   flags             NVFP4_GEMM_* kernel choice.
+ * Shapes: m >= 1, n a multiple of 16, k a multiple of 32, all < 2^31.
+ * The BF16 output is the round-to-nearest-even BF16 of the FP32 output of the
+ * same call configuration.  Results are deterministic (no atomics).
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
+                        const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs, int nsegs,
+                        void* c, nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, uint32_t flags,
+                        void* stream);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics.
+ * ---------------------------------------------------------------------- */
+
+/* Text of the last error returned on the calling thread ("" if none). */
+NVFP4_API const char* nvfp4_get_last_error_string(void);
+
+/* Synchronises `stream`, reads and clears the device status word that bounded
+ * waits set when they run out.  Returns NVFP4_ERR_TIMEOUT if any did (the
+ * kernel that timed out returned early and its outputs are undefined),
+ * NVFP4_ERR_CUDA if the synchronisation failed, NVFP4_OK otherwise. */
+NVFP4_API nvfp4_status nvfp4_check_device_status(void* stream);
+
+/* Enqueues a one-thread kernel that waits on an mbarrier nobody arrives at,
+ * for at most `limit_cycles` SM clock cycles, then records a timeout and
+ * returns.  Lets tests exercise the timeout reporting without a fault. */
+NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+NVFP4_API int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

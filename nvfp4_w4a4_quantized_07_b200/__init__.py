@@ -1,1 +1,240 @@
-"""NVFP4 W4A4 linear layers for B200 (sm_100a): Python binding of libnvfp4."""
+"""NVFP4 W4A4 linear layers for B200 (sm_100a): Python binding of libnvfp4.
+
+Argument marshalling only.  Every step of the path (amax, block quantisation,
+the block-scaled GEMM and its per-module scale epilogue) runs in the CUDA
+kernels behind the C ABI declared in ``include/nvfp4.h``; PyTorch supplies
+device memory and the current stream.  There is no CPU fallback: if
+``libnvfp4.so`` is missing or cannot be loaded every call raises.
+
+The raw C entry points are available under their C names
+(``nvfp4_quantize_weight``, ``nvfp4_quantize_act``, ``nvfp4_gemm``, ...) on
+the object returned by :func:`load`; the helpers below wrap them for torch
+tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+NVFP4_IN_BF16, NVFP4_IN_FP32 = 0, 1
+NVFP4_OUT_BF16, NVFP4_OUT_FP32 = 0, 1
+NVFP4_GEMM_AUTO, NVFP4_GEMM_FORCE_LARGE, NVFP4_GEMM_FORCE_DECODE = 0, 1, 2
+NVFP4_MAX_SEGMENTS = 16
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA", 5: "TIMEOUT",
+                6: "WORKSPACE"}
+EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
+            "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_get_last_error_string",
+            "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout", "nvfp4_version")
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, call: str, status: int, detail: str):
+        super().__init__(f"{call}: {STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("col_begin", ctypes.c_int64), ("col_end", ctypes.c_int64), ("w_global_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load():
+    """Load ``libnvfp4.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise NVFP4Error("load", 4, f"{LIB_PATH} is not built; run `python -m nvfp4_w4a4_quantized_07_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, SZ, U32, INT = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_int
+    L.nvfp4_sf_bytes.argtypes = [I64, I64]
+    L.nvfp4_sf_bytes.restype = SZ
+    L.nvfp4_sf_offset.argtypes = [I64, I64, I64]
+    L.nvfp4_sf_offset.restype = I64
+    L.nvfp4_quant_workspace_size.argtypes = []
+    L.nvfp4_quant_workspace_size.restype = SZ
+    L.nvfp4_gemm_workspace_size.argtypes = [I64, I64, I64, U32]
+    L.nvfp4_gemm_workspace_size.restype = SZ
+    L.nvfp4_quantize_weight.argtypes = [P, INT, I64, I64, I64, I64, I64, P, P, P, P, P, SZ, P]
+    L.nvfp4_quantize_weight.restype = INT
+    L.nvfp4_quantize_act.argtypes = [P, INT, I64, I64, I64, P, P, P, P, P, SZ, P]
+    L.nvfp4_quantize_act.restype = INT
+    L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
+    L.nvfp4_gemm.restype = INT
+    L.nvfp4_get_last_error_string.argtypes = []
+    L.nvfp4_get_last_error_string.restype = ctypes.c_char_p
+    L.nvfp4_check_device_status.argtypes = [P]
+    L.nvfp4_check_device_status.restype = INT
+    L.nvfp4_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
+    L.nvfp4_selftest_wait_timeout.restype = INT
+    L.nvfp4_version.argtypes = []
+    L.nvfp4_version.restype = INT
+    _lib = L
+    return L
+
+
+def _check(call: str, status: int):
+    if status != 0:
+        raise NVFP4Error(call, status, load().nvfp4_get_last_error_string().decode())
+
+
+def _stream(device=None):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _in_dtype(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return NVFP4_IN_BF16
+    if t.dtype == torch.float32:
+        return NVFP4_IN_FP32
+    raise TypeError(f"NVFP4 inputs must be bfloat16 or float32, got {t.dtype}")
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libnvfp4 operates on CUDA tensors only")
+
+
+def sf_bytes(rows: int, k: int) -> int:
+    return int(load().nvfp4_sf_bytes(rows, k))
+
+
+def sf_offset(row: int, kblock: int, k: int) -> int:
+    return int(load().nvfp4_sf_offset(row, kblock, k))
+
+
+def quant_workspace(device) -> "torch.Tensor":
+    import torch
+    return torch.zeros(load().nvfp4_quant_workspace_size(), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class QuantizedActivation:
+    q: "torch.Tensor"       # m x k/2 uint8
+    sf: "torch.Tensor"      # tiled scales, uint8
+    scale: "torch.Tensor"   # 1-element float32 device tensor (s_ga)
+    m: int
+    k: int
+
+
+@dataclass
+class FusedWeight:
+    q: "torch.Tensor"       # n x k/2 uint8
+    sf: "torch.Tensor"      # tiled scales, uint8
+    segments: list          # [(col_begin, col_end, w_global_scale)]
+    n: int
+    k: int
+
+
+def quantize_act(a, act_scale=None, workspace=None, out: QuantizedActivation | None = None) -> QuantizedActivation:
+    """On-the-fly activation quantisation (``nvfp4_quantize_act``).
+
+    ``act_scale``: 1-element float32 CUDA tensor holding a calibrated decode
+    scale (static mode) or ``None`` (dynamic: amax/2688 computed on device).
+    """
+    import torch
+    _require_cuda(a, act_scale)
+    if a.dim() != 2 or a.stride(1) != 1:
+        raise ValueError("activations must be a 2-D tensor with unit column stride")
+    m, k = a.shape
+    L = load()
+    if out is None:
+        out = QuantizedActivation(
+            q=torch.empty((m, k // 2), dtype=torch.uint8, device=a.device),
+            sf=torch.empty(max(L.nvfp4_sf_bytes(m, k), 1), dtype=torch.uint8, device=a.device),
+            scale=torch.empty(1, dtype=torch.float32, device=a.device), m=m, k=k)
+    if act_scale is None and workspace is None:
+        workspace = quant_workspace(a.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("nvfp4_quantize_act", L.nvfp4_quantize_act(
+        _ptr(a), _in_dtype(a), m, k, a.stride(0), _ptr(act_scale), _ptr(out.scale), _ptr(out.q), _ptr(out.sf),
+        _ptr(workspace), ws_bytes, _stream(a.device)))
+    return out
+
+
+def quantize_weight(modules, global_scales=None, workspace=None) -> FusedWeight:
+    """Quantise separately calibrated modules into one fused weight
+    (``nvfp4_quantize_weight`` once per module).  ``global_scales[i]`` (a
+    Python float) fixes module i's decode scale; ``None`` computes amax/2688
+    on the device (the call then synchronises to return it)."""
+    import torch
+    modules = list(modules)
+    if not modules:
+        raise ValueError("need at least one module")
+    k = modules[0].shape[1]
+    device = modules[0].device
+    n_total = sum(w.shape[0] for w in modules)
+    L = load()
+    q = torch.empty((n_total, k // 2), dtype=torch.uint8, device=device)
+    sf = torch.empty(max(L.nvfp4_sf_bytes(n_total, k), 1), dtype=torch.uint8, device=device)
+    if workspace is None:
+        workspace = quant_workspace(device)
+    segs = []
+    off = 0
+    for i, w in enumerate(modules):
+        _require_cuda(w)
+        if w.dim() != 2 or w.shape[1] != k or w.stride(1) != 1:
+            raise ValueError("every module must be a 2-D n_i x k tensor with unit column stride")
+        n = w.shape[0]
+        given = None if global_scales is None or global_scales[i] is None else ctypes.c_float(global_scales[i])
+        got = ctypes.c_float(0.0)
+        _check("nvfp4_quantize_weight", L.nvfp4_quantize_weight(
+            _ptr(w), _in_dtype(w), n, k, w.stride(0), off, n_total,
+            None if given is None else ctypes.byref(given), _ptr(q), _ptr(sf), ctypes.byref(got),
+            _ptr(workspace), workspace.numel(), _stream(device)))
+        segs.append((off, off + n, float(got.value)))
+        off += n
+    return FusedWeight(q=q, sf=sf, segments=segs, n=n_total, k=k)
+
+
+def segment_array(segments):
+    arr = (Segment * len(segments))()
+    for i, (b, e, s) in enumerate(segments):
+        arr[i].col_begin, arr[i].col_end, arr[i].w_global_scale = b, e, s
+    return arr
+
+
+def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NVFP4_GEMM_AUTO,
+         segments=None, out=None):
+    """``C = nvfp4_gemm(a, w)``: m x n output, BF16 by default.  ``segments``
+    overrides the fused weight's own segment table."""
+    import torch
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if a.k != w.k:
+        raise ValueError("K mismatch between activations and weight")
+    segments = w.segments if segments is None else segments
+    if out is None:
+        out = torch.empty((a.m, w.n), dtype=out_dtype, device=a.q.device)
+    odt = {torch.bfloat16: NVFP4_OUT_BF16, torch.float32: NVFP4_OUT_FP32}[out.dtype]
+    arr = segment_array(segments)
+    L = load()
+    _check("nvfp4_gemm", L.nvfp4_gemm(
+        _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
+        _ptr(out), odt, out.stride(0), None, 0, flags, _stream(out.device)))
+    return out
+
+
+def linear(a, w: FusedWeight, act_scale=None, out_dtype=None, flags: int = NVFP4_GEMM_AUTO):
+    """One W4A4 linear layer: quantise ``a`` on the fly, then the fused GEMM."""
+    return gemm(quantize_act(a, act_scale), w, out_dtype=out_dtype, flags=flags)
+
+
+def check_device_status(device=None):
+    _check("nvfp4_check_device_status", load().nvfp4_check_device_status(_stream(device)))
+
+
+def version() -> int:
+    return int(load().nvfp4_version())

@@ -1,0 +1,53 @@
+"""Build libnvfp4.so in-tree with nvcc for sm_100a.
+
+Usage: ``python -m nvfp4_w4a4_quantized_07_b200.build [--verbose-ptxas]``.
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+LIB = os.path.join(PKG, "libnvfp4.so")
+SOURCES = [os.path.join(CSRC, "nvfp4_lib.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quant.cuh", "gemm.cuh")] + \
+    [os.path.join(ROOT, "include", "nvfp4.h")]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def command(verbose_ptxas: bool = False) -> list:
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+           "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+           "-ftz=false", "-prec-div=true", "-prec-sqrt=true", "-fmad=true",
+           "-I" + os.path.join(ROOT, "include"), "-o", LIB] + SOURCES + ["-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+    if verbose_ptxas:
+        cmd.insert(1, "-Xptxas=-v")
+    return cmd
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(d) <= t for d in DEPS)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    if force or verbose_ptxas or not up_to_date():
+        subprocess.run(command(verbose_ptxas), check=True)
+    return LIB
+
+
+if __name__ == "__main__":
+    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
+    print(LIB)

@@ -1,0 +1,453 @@
+// libnvfp4: the C ABI declared in include/nvfp4.h.  Argument validation, TMA
+// descriptor creation and kernel launches; all arithmetic runs in the kernels
+// of quant.cuh and gemm.cuh.  Single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nvfp4.h"
+#include "gemm.cuh"
+#include "quant.cuh"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+thread_local char g_err[512] = "";
+
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+nvfp4_status ok()
+{
+    g_err[0] = '\0';
+    return NVFP4_OK;
+}
+
+#define NVFP4_CUDA_TRY(expr)                                                                         \
+    do {                                                                                            \
+        cudaError_t e_ = (expr);                                                                    \
+        if (e_ != cudaSuccess) return fail(NVFP4_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+    } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t pad_to(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// ---------------------------------------------------------------------------
+// Per-device state: SM count and one-time kernel attribute setup.
+// ---------------------------------------------------------------------------
+struct DeviceState {
+    bool ready = false;
+    int sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+nvfp4_status device_state(DeviceState** out)
+{
+    int dev = 0;
+    NVFP4_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceState& d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+        NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+        if (major != 10 || minor != 0)
+            return fail(NVFP4_ERR_UNSUPPORTED, "device %d is sm_%d%d; libnvfp4 is built for sm_100a only", dev, major,
+                        minor);
+        NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            large::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            decode::Layout<16>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            decode::Layout<32>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            decode::Layout<64>::SMEM_BYTES));
+        d.ready = true;
+    }
+    *out = &d;
+    return NVFP4_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link-time libcuda).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+nvfp4_status encode_fp4_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t k, int box_rows)
+{
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (g_encode == nullptr) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    // Packed FP4 viewed as bytes: dim 0 = K/2 bytes (contiguous), dim 1 = rows.
+    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Quantisation launch shared by the activation and weight entry points.
+// ---------------------------------------------------------------------------
+nvfp4_status check_quant_input(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t k, int64_t ld,
+                               const char* what)
+{
+    if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32) return fail(NVFP4_ERR_INVALID_ARG, "%s: bad input dtype", what);
+    if (rows < 0 || k <= 0 || k % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "%s: need rows >= 0 and k a positive multiple of 32 (rows=%lld k=%lld)",
+                    what, (long long)rows, (long long)k);
+    if (rows >= (1ll << 31) || k >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "%s: dimension >= 2^31", what);
+    if (ld < k) return fail(NVFP4_ERR_INVALID_ARG, "%s: leading dimension %lld < k %lld", what, (long long)ld,
+                            (long long)k);
+    const int64_t esz = dt == NVFP4_IN_FP32 ? 4 : 2;
+    if (rows > 0 && x == nullptr) return fail(NVFP4_ERR_INVALID_ARG, "%s: input pointer is NULL", what);
+    if (!aligned16(x) || (ld * esz) % 16 != 0)
+        return fail(NVFP4_ERR_ALIGNMENT, "%s: input rows must start on 16-byte boundaries", what);
+    return NVFP4_OK;
+}
+
+nvfp4_status launch_amax(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t k, int64_t ld, void* ws,
+                         cudaStream_t s, int sms)
+{
+    NVFP4_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(unsigned int), s));
+    if (rows == 0) return NVFP4_OK;
+    const int64_t vec = dt == NVFP4_IN_FP32 ? 4 : 8;
+    const int64_t total = rows * (k / vec);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+    amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, rows, k, ld, dt == NVFP4_IN_FP32,
+                                                  static_cast<unsigned int*>(ws));
+    NVFP4_CUDA_TRY(cudaGetLastError());
+    return NVFP4_OK;
+}
+
+nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s)
+{
+    const int64_t segs = (p.k + 255) / 256;
+    const int64_t units = p.sf_rows_end * segs;
+    if (units == 0) return NVFP4_OK;
+    const int64_t warps = (units + kQuantUnits - 1) / kQuantUnits;
+    const int64_t blocks = (warps + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
+    if (blocks >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "quantise: tensor too large");
+    quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(p);
+    NVFP4_CUDA_TRY(cudaGetLastError());
+    return NVFP4_OK;
+}
+
+nvfp4_status check_segments(const nvfp4_segment* segs, int nsegs, int64_t n, SegTable* out)
+{
+    if (segs == nullptr || nsegs < 1 || nsegs > NVFP4_MAX_SEGMENTS)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm: need 1..%d segments (got %d)", NVFP4_MAX_SEGMENTS, nsegs);
+    int64_t expect = 0;
+    out->count = nsegs;
+    for (int i = 0; i < nsegs; ++i) {
+        const nvfp4_segment& g = segs[i];
+        if (g.col_begin != expect)
+            return fail(NVFP4_ERR_INVALID_ARG, "gemm: segment %d starts at %lld, expected %lld (sorted, contiguous)", i,
+                        (long long)g.col_begin, (long long)expect);
+        if (g.col_end <= g.col_begin)
+            return fail(NVFP4_ERR_INVALID_ARG, "gemm: segment %d is empty or reversed", i);
+        if (g.col_end % 16 != 0)
+            return fail(NVFP4_ERR_INVALID_ARG, "gemm: segment %d ends at %lld, not a multiple of 16", i,
+                        (long long)g.col_end);
+        if (!(g.w_global_scale > 0.0f) || !std::isfinite(g.w_global_scale))
+            return fail(NVFP4_ERR_INVALID_ARG, "gemm: segment %d scale must be positive and finite", i);
+        out->end[i] = (int)g.col_end;
+        out->scale[i] = g.w_global_scale;
+        expect = g.col_end;
+    }
+    for (int i = nsegs; i < kMaxSegments; ++i) {
+        out->end[i] = (int)n;
+        out->scale[i] = out->scale[nsegs - 1];
+    }
+    if (expect != n)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm: segments cover [0, %lld), expected [0, %lld)", (long long)expect,
+                    (long long)n);
+    return NVFP4_OK;
+}
+
+template <int BT>
+nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, GemmParams p, int w_tiles, cudaStream_t s)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)w_tiles, (unsigned)p.splits, 1);
+    cfg.blockDim = dim3(decode::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = decode::Layout<BT>::SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (unsigned)p.splits;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT>, ta, tw, p));
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k)
+{
+    if (rows < 0 || k <= 0 || k % 16 != 0) return 0;
+    return (size_t)(pad_to(rows, 128) * pad_to(k / 16, 4));
+}
+
+int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k)
+{
+    if (row < 0 || k <= 0 || k % 16 != 0 || kblock < 0 || kblock >= pad_to(k / 16, 4)) return -1;
+    const int64_t katoms = pad_to(k / 16, 4) / 4;
+    return ((row / 128) * katoms + kblock / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + kblock % 4;
+}
+
+size_t nvfp4_quant_workspace_size(void) { return 256; }
+
+size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t, uint32_t) { return 0; }
+
+const char* nvfp4_get_last_error_string(void) { return g_err; }
+
+int nvfp4_version(void) { return kVersion; }
+
+nvfp4_status nvfp4_quantize_act(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                const float* act_scale_dev, float* act_scale_out_dev, uint8_t* a_q, uint8_t* a_sf,
+                                void* workspace, size_t ws_bytes, void* stream)
+{
+    nvfp4_status st = check_quant_input(a, dt, m, k, lda, "quantize_act");
+    if (st != NVFP4_OK) return st;
+    if (m > 0 && (a_q == nullptr || a_sf == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "quantize_act: a_q / a_sf is NULL");
+    if (!aligned16(a_q) || !aligned16(a_sf)) return fail(NVFP4_ERR_ALIGNMENT, "quantize_act: outputs not 16-byte aligned");
+    const bool dynamic = act_scale_dev == nullptr;
+    if (dynamic) {
+        if (act_scale_out_dev == nullptr)
+            return fail(NVFP4_ERR_INVALID_ARG, "quantize_act: dynamic mode needs act_scale_out_dev");
+        if (workspace == nullptr || ws_bytes < nvfp4_quant_workspace_size())
+            return fail(NVFP4_ERR_WORKSPACE, "quantize_act: dynamic mode needs %zu bytes of workspace",
+                        nvfp4_quant_workspace_size());
+        if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "quantize_act: workspace not 16-byte aligned");
+    }
+    if (m == 0) return ok();
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dynamic && (st = launch_amax(a, dt, m, k, lda, workspace, s, dev->sms)) != NVFP4_OK) return st;
+    QuantParams p = {};
+    p.x = a;
+    p.rows = m;
+    p.k = k;
+    p.ldx = lda;
+    p.in_fp32 = dt == NVFP4_IN_FP32;
+    p.q = a_q;
+    p.sf = a_sf;
+    p.row_offset = 0;
+    p.sf_rows_end = pad_to(m, 128);
+    p.scale_mode = dynamic ? kScaleFromAmax : kScaleDevice;
+    p.scale_ptr = dynamic ? static_cast<const float*>(workspace) : act_scale_dev;
+    p.scale_out = act_scale_out_dev;
+    if ((st = launch_quant(p, s)) != NVFP4_OK) return st;
+    return ok();
+}
+
+nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_in_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                                   int64_t row_offset, int64_t n_total, const float* global_scale_in,
+                                   uint8_t* w_q, uint8_t* w_sf, float* global_scale_out, void* workspace,
+                                   size_t ws_bytes, void* stream)
+{
+    nvfp4_status st = check_quant_input(w, dt, n, k, ldw, "quantize_weight");
+    if (st != NVFP4_OK) return st;
+    if (row_offset < 0 || n_total < row_offset + n || n_total >= (1ll << 31))
+        return fail(NVFP4_ERR_INVALID_ARG, "quantize_weight: rows [%lld, %lld) do not fit in n_total %lld",
+                    (long long)row_offset, (long long)(row_offset + n), (long long)n_total);
+    if (n > 0 && (w_q == nullptr || w_sf == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "quantize_weight: w_q / w_sf is NULL");
+    if (!aligned16(w_q) || !aligned16(w_sf))
+        return fail(NVFP4_ERR_ALIGNMENT, "quantize_weight: outputs not 16-byte aligned");
+    const bool computed = global_scale_in == nullptr;
+    if (computed) {
+        if (global_scale_out == nullptr)
+            return fail(NVFP4_ERR_INVALID_ARG, "quantize_weight: computed scale needs global_scale_out");
+        if (workspace == nullptr || ws_bytes < nvfp4_quant_workspace_size())
+            return fail(NVFP4_ERR_WORKSPACE, "quantize_weight: computing the scale needs %zu bytes of workspace",
+                        nvfp4_quant_workspace_size());
+        if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "quantize_weight: workspace not 16-byte aligned");
+    } else if (!(*global_scale_in > 0.0f) || !std::isfinite(*global_scale_in)) {
+        return fail(NVFP4_ERR_INVALID_ARG, "quantize_weight: global scale must be positive and finite");
+    }
+    const bool owns_tail = row_offset + n == n_total;
+    const int64_t sf_rows_end = owns_tail ? pad_to(n_total, 128) - row_offset : n;
+    if (sf_rows_end == 0) {
+        if (computed) *global_scale_out = 1.0f;
+        return ok();
+    }
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* ws_f = static_cast<float*>(workspace);
+    if (computed && (st = launch_amax(w, dt, n, k, ldw, workspace, s, dev->sms)) != NVFP4_OK) return st;
+    QuantParams p = {};
+    p.x = w;
+    p.rows = n;
+    p.k = k;
+    p.ldx = ldw;
+    p.in_fp32 = dt == NVFP4_IN_FP32;
+    p.q = w_q;
+    p.sf = w_sf;
+    p.row_offset = row_offset;
+    p.sf_rows_end = sf_rows_end;
+    if (computed) {
+        p.scale_mode = kScaleFromAmax;
+        p.scale_ptr = ws_f;
+        p.scale_out = ws_f + 1;
+    } else {
+        p.scale_mode = kScaleValue;
+        p.scale_value = *global_scale_in;
+    }
+    if ((st = launch_quant(p, s)) != NVFP4_OK) return st;
+    if (computed) {
+        NVFP4_CUDA_TRY(cudaMemcpyAsync(global_scale_out, ws_f + 1, sizeof(float), cudaMemcpyDeviceToHost, s));
+        NVFP4_CUDA_TRY(cudaStreamSynchronize(s));
+    } else if (global_scale_out != nullptr) {
+        *global_scale_out = *global_scale_in;
+    }
+    return ok();
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
+                        const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs, int nsegs,
+                        void* c, nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, uint32_t flags,
+                        void* stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (m < 0 || n <= 0 || k <= 0 || n % 16 != 0 || k % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm: need m >= 0, n a positive multiple of 16, k a positive multiple of 32 "
+                                           "(m=%lld n=%lld k=%lld)", (long long)m, (long long)n, (long long)k);
+    if (m >= (1ll << 31) || n >= (1ll << 31) || k >= (1ll << 31))
+        return fail(NVFP4_ERR_UNSUPPORTED, "gemm: dimension >= 2^31");
+    if (odt != NVFP4_OUT_BF16 && odt != NVFP4_OUT_FP32) return fail(NVFP4_ERR_INVALID_ARG, "gemm: bad output dtype");
+    if (flags > NVFP4_GEMM_FORCE_DECODE) return fail(NVFP4_ERR_INVALID_ARG, "gemm: unknown flags 0x%x", flags);
+    if (ldc < n) return fail(NVFP4_ERR_INVALID_ARG, "gemm: ldc %lld < n %lld", (long long)ldc, (long long)n);
+    SegTable table;
+    nvfp4_status st = check_segments(segs, nsegs, n, &table);
+    if (st != NVFP4_OK) return st;
+    if (m > 0 && (a_q == nullptr || a_sf == nullptr || act_scale_dev == nullptr || w_q == nullptr ||
+                  w_sf == nullptr || c == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm: NULL operand pointer");
+    const int64_t osz = odt == NVFP4_OUT_FP32 ? 4 : 2;
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(c) ||
+        (ldc * osz) % 16 != 0)
+        return fail(NVFP4_ERR_ALIGNMENT, "gemm: operands and output rows must be 16-byte aligned");
+    const bool use_decode = flags == NVFP4_GEMM_FORCE_DECODE || (flags == NVFP4_GEMM_AUTO && m <= 64);
+    if (use_decode && m > 64) return fail(NVFP4_ERR_UNSUPPORTED, "gemm: the decode kernel handles m <= 64");
+    if (m == 0) return ok();
+
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    GemmParams p = {};
+    p.m = (int)m;
+    p.n = (int)n;
+    p.k = (int)k;
+    p.a_sf = a_sf;
+    p.w_sf = w_sf;
+    p.act_scale = act_scale_dev;
+    p.c = c;
+    p.ldc = ldc;
+    p.out_fp32 = odt == NVFP4_OUT_FP32;
+    p.segs = table;
+    p.katoms = (int)(pad_to(k / 16, 4) / 4);
+    p.k_tiles = (int)((k + 255) / 256);
+    p.a_rowblocks = (int)((m + 127) / 128);
+    p.w_rowblocks = (int)((n + 127) / 128);
+    p.splits = 1;
+
+    CUtensorMap ta, tw;
+    if (!use_decode) {
+        p.m_tiles = (int)((m + large::BM - 1) / large::BM);
+        p.n_tiles = (int)((n + large::BN - 1) / large::BN);
+        if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
+        if ((st = encode_fp4_map(&tw, w_q, n, k, large::BN)) != NVFP4_OK) return st;
+        const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+        const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
+        gemm_large_kernel<<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, p);
+        NVFP4_CUDA_TRY(cudaGetLastError());
+        return ok();
+    }
+
+    const int bt = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
+    const int w_tiles = (int)((n + decode::BW - 1) / decode::BW);
+    int splits = (2 * dev->sms) / w_tiles;
+    if (splits > 8) splits = 8;
+    if (splits > p.k_tiles) splits = p.k_tiles;
+    if (splits < 1) splits = 1;
+    p.splits = splits;
+    p.m_tiles = 1;
+    p.n_tiles = w_tiles;
+    if ((st = encode_fp4_map(&ta, a_q, m, k, bt)) != NVFP4_OK) return st;
+    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BW)) != NVFP4_OK) return st;
+    if (bt == 16) st = launch_decode<16>(ta, tw, p, w_tiles, s);
+    else if (bt == 32) st = launch_decode<32>(ta, tw, p, w_tiles, s);
+    else st = launch_decode<64>(ta, tw, p, w_tiles, s);
+    if (st != NVFP4_OK) return st;
+    return ok();
+}
+
+nvfp4_status nvfp4_check_device_status(void* stream)
+{
+    NVFP4_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    unsigned int v = 0;
+    NVFP4_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_device_status, sizeof v));
+    if (v != 0) {
+        const unsigned int zero = 0;
+        NVFP4_CUDA_TRY(cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero));
+        return fail(NVFP4_ERR_TIMEOUT, "a bounded wait inside a kernel ran out (status 0x%x)", v);
+    }
+    return ok();
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(long long limit_cycles, void* stream)
+{
+    if (limit_cycles <= 0 || limit_cycles > kWaitCycles)
+        return fail(NVFP4_ERR_INVALID_ARG, "selftest: limit must be in (0, %lld] cycles", kWaitCycles);
+    selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    NVFP4_CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+"""The C-ABI library: it loads, exports every symbol include/nvfp4.h declares,
+its layout helpers agree with the oracle's independent index map, and argument
+errors come back as status codes before any CUDA call (so these run without a
+GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import nvfp4_w4a4_quantized_07_b200 as nv
+from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nvbuild.build()
+    return nv.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_gemm"):
+        assert n in names
+    assert set(names) == set(nv.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version(lib):
+    assert lib.nvfp4_version() >= 100
+
+
+def test_sf_layout_helpers_match_oracle_map(lib):
+    for rows, k in [(1, 32), (64, 256), (129, 288), (300, 320), (12384, 5120)]:
+        assert lib.nvfp4_sf_bytes(rows, k) == oracle.sf_tiled_bytes(rows, k)
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        k = int(rng.integers(1, 400)) * 16
+        row = int(rng.integers(0, 5000))
+        kb = int(rng.integers(0, k // 16))
+        assert lib.nvfp4_sf_offset(row, kb, k) == oracle.sf_tiled_offset(row, kb, k)
+    assert lib.nvfp4_sf_offset(0, 0, 30) == -1
+    assert lib.nvfp4_sf_offset(-1, 0, 32) == -1
+    assert lib.nvfp4_sf_bytes(4, 24) == 0
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+FAKE = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_quantize_act_argument_errors(lib):
+    ws = ctypes.c_void_p(0x20000)
+    st = lib.nvfp4_quantize_act(FAKE, 0, 8, 48, 48, None, FAKE, FAKE, FAKE, ws, 256, None)
+    assert st == 1 and b"multiple of 32" in lib.nvfp4_get_last_error_string()
+    assert lib.nvfp4_quantize_act(FAKE, 7, 8, 64, 64, FAKE, None, FAKE, FAKE, None, 0, None) == 1   # bad dtype
+    assert lib.nvfp4_quantize_act(FAKE, 0, 8, 64, 32, FAKE, None, FAKE, FAKE, None, 0, None) == 1   # lda < k
+    assert lib.nvfp4_quantize_act(None, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, None, 0, None) == 1   # null input
+    assert lib.nvfp4_quantize_act(MISALIGNED, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, None, 0, None) == 3
+    assert lib.nvfp4_quantize_act(FAKE, 0, 8, 64, 68, FAKE, None, FAKE, FAKE, None, 0, None) == 3   # row pitch
+    # dynamic mode needs an output scale and a workspace
+    assert lib.nvfp4_quantize_act(FAKE, 0, 8, 64, 64, None, None, FAKE, FAKE, ws, 256, None) == 1
+    assert lib.nvfp4_quantize_act(FAKE, 0, 8, 64, 64, None, FAKE, FAKE, FAKE, None, 0, None) == 6
+    assert lib.nvfp4_quantize_act(FAKE, 0, 8, 64, 64, None, FAKE, FAKE, FAKE, ws, 16, None) == 6
+    # empty input is a no-op that needs no device
+    assert lib.nvfp4_quantize_act(FAKE, 0, 0, 64, 64, FAKE, None, FAKE, FAKE, None, 0, None) == 0
+
+
+def test_quantize_weight_argument_errors(lib):
+    one = ctypes.c_float(1.0)
+    bad = ctypes.c_float(-1.0)
+    nan = ctypes.c_float(float("nan"))
+    out = ctypes.c_float(0)
+    f = lib.nvfp4_quantize_weight
+    assert f(FAKE, 0, 16, 64, 64, 10, 20, ctypes.byref(one), FAKE, FAKE, None, None, 0, None) == 1  # rows overflow
+    assert f(FAKE, 0, 16, 64, 64, -1, 20, ctypes.byref(one), FAKE, FAKE, None, None, 0, None) == 1
+    assert f(FAKE, 0, 16, 64, 64, 0, 16, ctypes.byref(bad), FAKE, FAKE, None, None, 0, None) == 1
+    assert f(FAKE, 0, 16, 64, 64, 0, 16, ctypes.byref(nan), FAKE, FAKE, None, None, 0, None) == 1
+    assert f(FAKE, 0, 16, 64, 64, 0, 16, None, FAKE, FAKE, None, FAKE, 256, None) == 1        # no scale out
+    assert f(FAKE, 0, 16, 64, 64, 0, 16, None, FAKE, FAKE, ctypes.byref(out), None, 0, None) == 6
+    assert f(FAKE, 0, 16, 64, 64, 0, 16, ctypes.byref(one), MISALIGNED, FAKE, None, None, 0, None) == 3
+
+
+def _segs(*triples):
+    return nv.segment_array(list(triples))
+
+
+def test_gemm_segment_table_errors(lib):
+    g = lib.nvfp4_gemm
+
+    def call(segs, n=64, nsegs=None):
+        nsegs = len(segs) if nsegs is None else nsegs
+        return g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, n, 64, segs, nsegs, FAKE, 0, n, None, 0, 0, None)
+
+    assert call(_segs((0, 32, 1.0), (40, 64, 1.0))) == 1          # gap
+    assert call(_segs((0, 48, 1.0), (32, 64, 1.0))) == 1          # overlap
+    assert call(_segs((32, 64, 1.0), (0, 32, 1.0))) == 1          # unsorted
+    assert call(_segs((0, 48, 1.0))) == 1                         # does not cover n
+    assert call(_segs((0, 24, 1.0), (24, 64, 1.0))) == 1          # boundary not a multiple of 16
+    assert call(_segs((0, 64, 0.0))) == 1                         # non-positive scale
+    assert call(_segs((0, 64, float("inf")))) == 1
+    assert call(_segs((0, 64, 1.0)), nsegs=0) == 1
+    many = _segs(*[(16 * i, 16 * (i + 1), 1.0) for i in range(17)])
+    assert call(many, n=17 * 16) == 1                             # more than 16 segments
+    assert b"segment" in lib.nvfp4_get_last_error_string()
+
+
+def test_gemm_shape_and_alignment_errors(lib):
+    g = lib.nvfp4_gemm
+    s = _segs((0, 64, 1.0))
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 48, s, 1, FAKE, 0, 64, None, 0, 0, None) == 1      # k % 32
+    s40 = _segs((0, 40, 1.0))
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 40, 64, s40, 1, FAKE, 0, 40, None, 0, 0, None) == 1    # n % 16
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 32, None, 0, 0, None) == 1      # ldc < n
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 5, 64, None, 0, 0, None) == 1      # out dtype
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, None, 0, 9, None) == 1      # flags
+    assert g(FAKE, FAKE, None, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None) == 1      # null scale
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, MISALIGNED, 0, 64, None, 0, 0, None) == 3
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 68, None, 0, 0, None) == 3     # row pitch
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 65, 64, 64, s, 1, FAKE, 0, 64, None, 0, 2, None) == 2     # decode m>64
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None) == 0      # empty
+
+
+def test_valid_call_without_a_gpu_fails_loudly(lib):
+    """With arguments that pass validation, a machine without a usable sm_100a
+    GPU gets NVFP4_ERR_CUDA / UNSUPPORTED, never a silent result."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    s = _segs((0, 64, 1.0))
+    st = lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None)
+    assert st in (2, 4)
+    assert lib.nvfp4_get_last_error_string()
