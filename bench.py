@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-gemm", action="store_true",
                     help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
+    ap.add_argument("--decode-case", default=None,
+                    help="time one decode GEMM only, e.g. m16_5120x5120 (for ncu captures)")
     return ap.parse_args()
 
 
@@ -174,7 +176,7 @@ def run_reference(args):
     s_ga = oracle.global_scale(a32)
     qmods = oracle.quantize_modules(p.modules)
     w_hat = oracle.fused_weight_hat(qmods)
-    rows = 8
+    rows = 256
     rng = np.random.default_rng(0)
 
     def step():
@@ -256,6 +258,9 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clocks:
+        # Busy the GPU while the host enqueues, so no host launch latency sits
+        # between a step's start event and its first kernel.
+        torch.cuda._sleep(2_000_000)
         for i in range(args.steps):
             step(events[i])
             flush.zero_()
@@ -310,9 +315,9 @@ def run_ours(args):
             **result,
         }
         if not args.profile_gemm and not args.no_cpu_baseline:
-            tf, dt, threads = time_oracle(p, rows=16, repeats=1)
+            tf, dt, threads = time_oracle(p, rows=2048, repeats=1)
             line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                    "sample": f"16 rows of A x all {p.n} columns (activation quantisation + "
+                                    "sample": f"2048 rows of A x all {p.n} columns (activation quantisation + "
                                               f"FP64 GEMM), {dt:.2f} s; weights quantised once, untimed"}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -340,6 +345,7 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
         e2e_step()
     n_e2e = max(3, min(args.steps, 10))
     torch.cuda.synchronize(device)
+    torch.cuda._sleep(1_000_000)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
@@ -358,6 +364,7 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
     for _ in range(3):
         nv.quantize_act(a_dev, workspace=ws, out=aq)
     flush.zero_()
+    torch.cuda._sleep(1_000_000)
     evs[0].record(stream)
     nv.quantize_act(a_dev, workspace=ws, out=aq)
     nv.gemm(aq, fw, out=c)
@@ -384,6 +391,7 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
                 times = []
                 for it in range(13):
                     flush.zero_()
+                    torch.cuda._sleep(400_000)       # keep host launch latency out of the events
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     e0.record(stream)
                     nv.gemm(aqd, fwd, out=cd)
@@ -402,10 +410,49 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
     return out
 
 
+def run_decode_case(args):
+    """One decode-shaped GEMM (``m<M>_<shape>``), L2 flushed before each launch."""
+    import torch
+
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+
+    m_str, shape = args.decode_case.split("_", 1)
+    m = int(m_str[1:])
+    nvbuild.build()
+    nv.load()
+    device = torch.device("cuda", 0)
+    p = synthetic.decode(m, shape)
+    fw = nv.quantize_weight([w.to(device) for w in p.modules])
+    aq = nv.quantize_act(p.a.to(device))
+    c = torch.empty((m, fw.n), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    times = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        torch.cuda._sleep(400_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nv.gemm(aq, fw, out=c)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    nbytes = fw.n * p.k // 2 + fw.n * p.k // 16 + m * p.k // 2 + m * p.k // 16 + m * fw.n * 2
+    print(json.dumps({"decode_case": args.decode_case, "us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9,
+                      "steps": args.steps}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode_case:
+        return run_decode_case(args)
     return run_ours(args)
 
 

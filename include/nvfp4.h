@@ -77,9 +77,10 @@ typedef struct {
 #define NVFP4_MAX_SEGMENTS 16
 
 /* nvfp4_gemm flags */
-#define NVFP4_GEMM_AUTO 0u          /* decode kernel for m <= 64, large kernel otherwise */
-#define NVFP4_GEMM_FORCE_LARGE 1u   /* always the persistent large-M kernel */
-#define NVFP4_GEMM_FORCE_DECODE 2u  /* always the split-K decode kernel (m <= 64) */
+#define NVFP4_GEMM_AUTO 0u              /* decode kernel for m <= 64, large kernel otherwise */
+#define NVFP4_GEMM_FORCE_LARGE 1u       /* the persistent large-M kernel (one CTA per SM, 128 x 256 tiles) */
+#define NVFP4_GEMM_FORCE_DECODE 2u      /* the split-K decode kernel (m <= 64) */
+#define NVFP4_GEMM_FORCE_LARGE_PAIR 3u  /* the large-M kernel on CTA pairs (cta_group::2, 256 x 256 tiles) */
 
 /* ------------------------------------------------------------------------
  * Layout helpers (pure host functions, no CUDA calls).

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 NVFP4_IN_BF16, NVFP4_IN_FP32 = 0, 1
 NVFP4_OUT_BF16, NVFP4_OUT_FP32 = 0, 1
-NVFP4_GEMM_AUTO, NVFP4_GEMM_FORCE_LARGE, NVFP4_GEMM_FORCE_DECODE = 0, 1, 2
+NVFP4_GEMM_AUTO, NVFP4_GEMM_FORCE_LARGE, NVFP4_GEMM_FORCE_DECODE, NVFP4_GEMM_FORCE_LARGE_PAIR = 0, 1, 2, 3
 NVFP4_MAX_SEGMENTS = 16
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA", 5: "TIMEOUT",
                 6: "WORKSPACE"}

@@ -91,8 +91,55 @@ __device__ __forceinline__ void store8(void* c, int64_t ldc, int out_fp32, int r
 }
 
 // ===========================================================================
-// Large-M kernel
+// Large-M kernel (one CTA per SM, 128 x 256 tiles, 256-deep K stages)
+//
+// Warp roles (16 warps):
+//   0      TMA producer: A/B tiles and the stage's scale atoms into a 4-stage ring
+//   1      MMA issuer: tcgen05 block-scaled MMAs (M=128, N=256, K=64)
+//   2      owns the TMEM allocation
+//   4..11  epilogue: drain the accumulator, scale by s_ga * s_gw[segment], store
+//   12..15 scale staging: read each stage's scale atoms from shared memory and
+//          write them into TMEM with tcgen05.st (one warp per 32-lane quadrant,
+//          every quadrant receiving the full atom), keeping the tensor pipe free
+//          for MMAs
+//
+// TMEM (512 columns): two 256-column accumulators overlapping by 96 columns,
+// ACC0 = [0, 256) and ACC1 = [160, 416), and two 48-column scale slots at
+// [416, 512).  Consecutive tiles alternate accumulators; the epilogue drains
+// the shared 96 columns first and releases them, so the next tile's MMAs start
+// while the rest of the previous tile is still being drained.
 // ===========================================================================
+// Drain one warp's 32 x 128 slice of an accumulator into scaled BF16 pairs,
+// 32 columns at a time starting with chunk ROT (compile-time so the results
+// stay in registers).  After the third chunk the warp optionally arrives on
+// `after3` (the columns shared with the other accumulator are then free).
+template <int ROT>
+__device__ __forceinline__ void drain_bf16(uint32_t taddr, int ncol0, float s_ga, const GemmParams& p,
+                                           uint64_t* after3, int lane, uint32_t (&packed)[4][16])
+{
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const int j = (ROT + jj) & 3;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + j * 32, v);
+        tmem_ld_wait();
+        if (jj == 2 && after3 != nullptr) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(after3);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int col = ncol0 + j * 32 + h * 16;
+            const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col < p.n ? col : p.n - 1));
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                packed[j][h * 8 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h * 16 + 2 * e]), alpha),
+                                                   __fmul_rn(__uint_as_float(v[h * 16 + 2 * e + 1]), alpha));
+        }
+    }
+}
+
 namespace large {
 constexpr int BM = 128, BN = 256, BK_BYTES = 128;  // BK = 256 FP4 values per stage
 constexpr int STAGES = 4;
@@ -106,13 +153,16 @@ constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int NUM_BARS = 2 * STAGES + 3;
+// full[S], empty[S], sf_ready[2], sf_free[2], acc_full[2], acc_empty[2], ovl_free, drain
+constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 2 + 1 + 1;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;  // + alignment slack
-constexpr int THREADS = 384;                          // 4 control warps + 8 epilogue warps
+constexpr int THREADS = 512;
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_SF = 256;                          // scale ring after the 256 accumulator columns
-constexpr int TMEM_SF_STAGE = 48;                     // 16 (A) + 32 (B) columns per stage
+constexpr int ACC1_COL = 160;                         // ACC0 at 0; overlap [160, 256)
+constexpr int SF_COL = 416;                           // two scale slots of 48 columns
+constexpr int SF_SLOT = 48;                           // 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
+static_assert(ACC1_COL + BN <= SF_COL && SF_COL + 2 * SF_SLOT <= TMEM_COLS, "TMEM budget");
 }  // namespace large
 
 __global__ void __launch_bounds__(large::THREADS, 1)
@@ -124,9 +174,12 @@ __global__ void __launch_bounds__(large::THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* empty = full + STAGES;
-    uint64_t* tmem_full = empty + STAGES;
-    uint64_t* tmem_empty = tmem_full + 1;
-    uint64_t* drain = tmem_empty + 1;
+    uint64_t* sf_ready = empty + STAGES;
+    uint64_t* sf_free = sf_ready + 2;
+    uint64_t* acc_full = sf_free + 2;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* ovl_free = acc_empty + 2;
+    uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
     const int warp = threadIdx.x >> 5;
@@ -140,8 +193,13 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 8);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sf_ready[i], 4);
+            mbar_init(&sf_free[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 8);
+        }
+        mbar_init(ovl_free, 4);
         mbar_init(drain, 1);
         fence_mbarrier_init();
     }
@@ -201,10 +259,325 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_nvf4(BM, BN);
+            int stage = 0, slot = 0;
+            uint32_t phase = 0, slot_phase = 0;
+            bool ok = true;
+            int i = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++i) {
+                const int b = i & 1;
+                // This accumulator's previous tile (i - 2) is fully drained, and
+                // the columns it shares with the other one are free (tile i - 1).
+                if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, kStatusTimeoutAccum) ||
+                    (i > 0 && !mbar_wait(ovl_free, (i - 1) & 1, kStatusTimeoutAccum))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem_base + (b ? ACC1_COL : 0);
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!mbar_wait(&sf_ready[slot], slot_phase, kStatusTimeoutFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
+                    const uint32_t sf_col = tmem_base + SF_COL + slot * SF_SLOT;
+                    const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
+                    const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
+                    for (int ks = 0; ks < nks; ++ks) {
+                        // 64 FP4 values = 32 bytes along K: +2 in the descriptor's 16-byte units.
+                        mma_nvf4(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0, sf_col + 4 * ks,
+                                 sf_col + 16 + 8 * ks);
+                    }
+                    mma_commit(&empty[stage]);
+                    mma_commit(&sf_free[slot]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                    if (++slot == 2) {
+                        slot = 0;
+                        slot_phase ^= 1;
+                    }
+                }
+                mma_commit(&acc_full[b]);
+            }
+            if (!ok) {
+                // After an abort, wait (bounded) until every MMA issued so far has
+                // finished before the CTA can free TMEM and leave.
+                mma_commit(drain);
+                mbar_wait(drain, 0, kStatusTimeoutDrain, kWaitCycles / 8);
+            }
+            (void)phase;
+        }
+        __syncwarp();
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ scale staging
+        // Quadrant q writes lanes 32q..32q+31; each lane l receives row l of every
+        // atom (16 bytes = the scales of rows l, l+32, l+64, l+96), which is the
+        // layout block-scaled MMAs read for both operands.
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, slot_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kt = 0; kt < p.k_tiles; ++kt) {
+                if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull) ||
+                    !mbar_wait(&sf_free[slot], slot_phase ^ 1, kStatusTimeoutFull)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE + lane * 16;
+                const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE + lane * 16;
+                uint32_t ra[16], rb[16], rc[16];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + ks * 512);
+                    ra[4 * ks] = a.x;
+                    ra[4 * ks + 1] = a.y;
+                    ra[4 * ks + 2] = a.z;
+                    ra[4 * ks + 3] = a.w;
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + ks * 512);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + ks * 512);
+                    uint32_t* d = ks < 2 ? rb : rc;
+                    const int o = (ks & 1) * 8;
+                    d[o] = b0.x;
+                    d[o + 1] = b0.y;
+                    d[o + 2] = b0.z;
+                    d[o + 3] = b0.w;
+                    d[o + 4] = b1.x;
+                    d[o + 5] = b1.y;
+                    d[o + 6] = b1.z;
+                    d[o + 7] = b1.w;
+                }
+                const uint32_t col = tmem_base + lane_base + SF_COL + slot * SF_SLOT;
+                tmem_st_32x32b_x16(col, ra);        // A: k-step ks at columns 4ks .. 4ks+3
+                tmem_st_32x32b_x16(col + 16, rb);   // B: k-step ks at columns 16+8ks .. 16+8ks+7
+                tmem_st_32x32b_x16(col + 32, rc);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[slot]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+                if (++slot == 2) {
+                    slot = 0;
+                    slot_phase ^= 1;
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 4;
+        const int quad = warp & 3;  // TMEM lanes this warp may access
+        const int half = ew >> 2;   // which 128 accumulator columns
+        const float s_ga = *p.act_scale;
+        int i = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+            const int b = i & 1;
+            const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
+            if (!mbar_wait(&acc_full[b], (i >> 1) & 1, kStatusTimeoutAccum)) break;
+            tc_fence_after();
+            const int row = mb * BM + quad * 32 + lane;
+            const int ncol0 = nb * BN + half * 128;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (b ? ACC1_COL : 0) + half * 128;
+            // The 96 columns shared with the other accumulator: ACC0's columns
+            // 160..255 (chunks 1-3 of half 1) or ACC1's columns 0..95 (chunks 0-2
+            // of half 0).  Their owners drain them first and release them.
+            const bool owns_overlap = half == (b == 0 ? 1 : 0);
+            const int first = (b == 0) ? 1 : 0;
+            if (!p.out_fp32) {
+                uint32_t packed[4][16];
+                if (owns_overlap && first == 1)
+                    drain_bf16<1>(taddr, ncol0, s_ga, p, ovl_free, lane, packed);
+                else
+                    drain_bf16<0>(taddr, ncol0, s_ga, p, owns_overlap ? ovl_free : nullptr, lane, packed);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+                if (row < p.m) {
+                    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = ncol0 + j * 32 + g * 8;
+                            if (col < p.n)
+                                *reinterpret_cast<uint4*>(crow + col) =
+                                    make_uint4(packed[j][4 * g], packed[j][4 * g + 1], packed[j][4 * g + 2],
+                                               packed[j][4 * g + 3]);
+                        }
+                }
+            } else {
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = owns_overlap ? (first + jj) & 3 : jj;
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + j * 32, v);
+                    tmem_ld_wait();
+                    if (owns_overlap && jj == 2) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(ovl_free);
+                    }
+                    if (jj == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[b]);
+                    }
+                    const int col0 = ncol0 + j * 32;
+                    if (row < p.m && col0 < p.n) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = col0 + 8 * g;
+                            if (col < p.n) {
+                                const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
+                                float o[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__uint_as_float(v[8 * g + e]), alpha);
+                                store8(p.c, p.ldc, 1, row, col, o);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ===========================================================================
+// Large-M kernel on CTA pairs (cta_group::2): a cluster of two CTAs on two SMs
+// computes a 256 x 256 tile with M = 256 MMAs.  Each CTA stages only its own
+// 128 rows of A and its own 128 rows of B (the pair's MMA reads both halves),
+// so each SM moves half the B bytes through shared memory per FLOP of the
+// single-CTA kernel; the even CTA issues the scale copies and MMAs for both.
+// Scale factors arrive by TMA too (3-D view: 512-byte atoms x K-atoms x
+// 128-row blocks), so out-of-range atoms are zero-filled by the copy engine.
+// ===========================================================================
+namespace pairk {
+constexpr int CTA_ROWS = 128, BN = 256, BK_BYTES = 128;
+constexpr int STAGES = 5;
+constexpr int KSTEPS = 4;
+constexpr int A_STAGE = CTA_ROWS * BK_BYTES;        // 16 KB: this CTA's half of the 256 A rows
+constexpr int B_STAGE = (BN / 2) * BK_BYTES;        // 16 KB: this CTA's half of the 256 B rows
+constexpr int SFA_STAGE = 4 * 512;                  // 4 atoms of this CTA's 128 A rows
+constexpr int SFB_STAGE = 2 * 4 * 512;              // all 256 B rows: 2 row blocks x 4 atoms
+constexpr uint32_t STAGE_TX = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int NUM_BARS = 2 * STAGES + 3;
+constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;
+constexpr int THREADS = 384;
+constexpr int TMEM_COLS = 512;
+constexpr int TMEM_SF = 256;
+constexpr int TMEM_SF_STAGE = 48;
+static_assert(TMEM_SF + STAGES * TMEM_SF_STAGE <= TMEM_COLS, "TMEM budget");
+}  // namespace pairk
+
+__global__ void __launch_bounds__(pairk::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfw,
+                     const __grid_constant__ GemmParams p)
+{
+    using namespace pairk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* drain = tmem_empty + 1;
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();     // 0: issues the pair's MMAs
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int num_tiles = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row tiles here
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tensor_map(&tmap_a);
+        prefetch_tensor_map(&tmap_w);
+        prefetch_tensor_map(&tmap_sfa);
+        prefetch_tensor_map(&tmap_sfw);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 16);  // 8 epilogue warps in each CTA of the pair
+        mbar_init(drain, 1);
+        fence_mbarrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(tmem_ptr, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    // Both CTAs' barriers exist before either CTA may signal the other's.
+    tc_fence_before();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_ptr;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
+                for (int kt = 0; kt < p.k_tiles; ++kt) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    // The stage's four copies of BOTH CTAs complete on the even CTA's barrier.
+                    const uint32_t bar0 = map_shared_rank(smem_u32(&full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_TX);
+                    tma_load_2d_pair(smem + OFF_A + stage * A_STAGE, &tmap_a, bar0, kt * BK_BYTES,
+                                     mb * 2 * CTA_ROWS + (int)rank * CTA_ROWS);
+                    tma_load_2d_pair(smem + OFF_B + stage * B_STAGE, &tmap_w, bar0, kt * BK_BYTES,
+                                     nb * BN + (int)rank * (BN / 2));
+                    tma_load_3d_pair(smem + OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar0, 0, kt * KSTEPS,
+                                     2 * mb + (int)rank);
+                    tma_load_3d_pair(smem + OFF_SFB + stage * SFB_STAGE, &tmap_sfw, bar0, 0, kt * KSTEPS, 2 * nb);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                const long long t0 = clock64();
+                while (clock64() - t0 < kWaitCycles / 64) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_nvf4(2 * CTA_ROWS, BN);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
                 if (!mbar_wait(tmem_empty, acc_phase ^ 1, kStatusTimeoutAccum)) {
                     ok = false;
                     break;
@@ -221,67 +594,100 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                     const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE;
                     const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE;
                     for (int ks = 0; ks < nks; ++ks) {
-                        tmem_cp_32x128b_x4(sf_col + 4 * ks, desc_sf_atom(sfa + ks * 512));
-                        tmem_cp_32x128b_x4(sf_col + 16 + 8 * ks, desc_sf_atom(sfb + ks * 512));
-                        tmem_cp_32x128b_x4(sf_col + 16 + 8 * ks + 4, desc_sf_atom(sfb + 2048 + ks * 512));
+                        tmem_cp_32x128b_x4_pair(sf_col + 4 * ks, desc_sf_atom(sfa + ks * 512));
+                        tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * ks, desc_sf_atom(sfb + ks * 512));
+                        tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * ks + 4, desc_sf_atom(sfb + 2048 + ks * 512));
                     }
                     const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
                     const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
-                    for (int ks = 0; ks < nks; ++ks) {
-                        // 64 FP4 values = 32 bytes along K: +2 in the descriptor's 16-byte units.
-                        mma_nvf4(tmem_base, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0,
-                                 sf_col + 4 * ks, sf_col + 16 + 8 * ks);
-                    }
-                    mma_commit(&empty[stage]);
+                    for (int ks = 0; ks < nks; ++ks)
+                        mma_nvf4_pair(tmem_base, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0,
+                                      sf_col + 4 * ks, sf_col + 16 + 8 * ks);
+                    mma_commit_pair(&empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
-                mma_commit(tmem_full);
+                mma_commit_pair(tmem_full, 0x3);
                 acc_phase ^= 1;
             }
             if (!ok) {
-                // After an abort, wait (bounded) until every MMA issued so far has
-                // finished before the CTA can free TMEM and leave.
-                mma_commit(drain);
+                mma_commit_pair(drain, 0x1);
                 mbar_wait(drain, 0, kStatusTimeoutDrain, kWaitCycles / 8);
             }
         }
         __syncwarp();
     } else if (warp >= 4) {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 4;
-        const int quad = warp & 3;  // TMEM lanes this warp may access
-        const int half = ew >> 2;   // which 128 accumulator columns
+        const int quad = warp & 3;
+        const int half = ew >> 2;
+        const uint32_t empty0 = map_shared_rank(smem_u32(tmem_empty), 0);
         uint32_t acc_phase = 0;
         const float s_ga = *p.act_scale;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        for (int tile = pair; tile < num_tiles; tile += npairs) {
             const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
             if (!mbar_wait(tmem_full, acc_phase, kStatusTimeoutAccum)) break;
             tc_fence_after();
-            const int row = mb * BM + quad * 32 + lane;
-            for (int j = 0; j < 4; ++j) {
-                const int lcol = half * 128 + j * 32;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quad * 32) << 16) + lcol, v);
-                tmem_ld_wait();
-                if (j == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(tmem_empty);
+            const int row = mb * 2 * CTA_ROWS + (int)rank * CTA_ROWS + quad * 32 + lane;
+            const int ncol0 = nb * BN + half * 128;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + half * 128;
+            if (!p.out_fp32) {
+                uint32_t packed[4][16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + j * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int col = ncol0 + j * 32 + h * 16;
+                        const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col < p.n ? col : p.n - 1));
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            packed[j][h * 8 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h * 16 + 2 * e]), alpha),
+                                                               __fmul_rn(__uint_as_float(v[h * 16 + 2 * e + 1]), alpha));
+                    }
                 }
-                const int col0 = nb * BN + lcol;
-                if (row < p.m && col0 < p.n) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty0);
+                if (row < p.m) {
+                    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int col = col0 + 8 * g;
-                        if (col < p.n) {
-                            const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
-                            float o[8];
+                    for (int j = 0; j < 4; ++j)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__uint_as_float(v[8 * g + e]), alpha);
-                            store8(p.c, p.ldc, p.out_fp32, row, col, o);
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = ncol0 + j * 32 + g * 8;
+                            if (col < p.n)
+                                *reinterpret_cast<uint4*>(crow + col) =
+                                    make_uint4(packed[j][4 * g], packed[j][4 * g + 1], packed[j][4 * g + 2],
+                                               packed[j][4 * g + 3]);
+                        }
+                }
+            } else {
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(taddr + j * 32, v);
+                    tmem_ld_wait();
+                    if (j == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(empty0);
+                    }
+                    const int col0 = ncol0 + j * 32;
+                    if (row < p.m && col0 < p.n) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = col0 + 8 * g;
+                            if (col < p.n) {
+                                const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
+                                float o[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__uint_as_float(v[8 * g + e]), alpha);
+                                store8(p.c, p.ldc, 1, row, col, o);
+                            }
                         }
                     }
                 }
@@ -290,11 +696,13 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         }
     }
 
+    // Neither CTA leaves (or frees TMEM) while the other may still signal it.
     tc_fence_before();
-    __syncthreads();
+    cluster_arrive_release();
+    cluster_wait_acquire();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 

@@ -76,6 +76,8 @@ nvfp4_status device_state(DeviceState** out)
         NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             large::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            pairk::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             decode::Layout<16>::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -116,6 +118,25 @@ nvfp4_status encode_fp4_map(CUtensorMap* map, const uint8_t* base, int64_t rows,
     return NVFP4_OK;
 }
 
+// Tiled scale buffer viewed as 32-bit words: dim 0 = the 128 words of one
+// 512-byte atom, dim 1 = K-atoms, dim 2 = 128-row blocks.  A box of
+// {128, 4, box_blocks} is one pipeline stage's scales; atoms past the end of
+// either dimension are zero-filled by the copy engine.
+nvfp4_status encode_sf_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t k, int box_blocks)
+{
+    const int64_t katoms = pad_to(k / 16, 4) / 4;
+    const int64_t blocks = (rows + 127) / 128;
+    const cuuint64_t dims[3] = {128u, (cuuint64_t)katoms, (cuuint64_t)blocks};
+    const cuuint64_t strides[2] = {512u, (cuuint64_t)(katoms * 512)};
+    const cuuint32_t box[3] = {128u, 4u, (cuuint32_t)box_blocks};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Quantisation launch shared by the activation and weight entry points.
 // ---------------------------------------------------------------------------
@@ -153,14 +174,22 @@ nvfp4_status launch_amax(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t
 
 nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s)
 {
-    const int64_t segs = (p.k + 255) / 256;
-    const int64_t units = p.sf_rows_end * segs;
-    if (units == 0) return NVFP4_OK;
-    const int64_t warps = (units + kQuantUnits - 1) / kQuantUnits;
-    const int64_t blocks = (warps + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
-    if (blocks >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "quantise: tensor too large");
-    quantize_kernel<<<(unsigned)blocks, kQuantThreads, 0, s>>>(p);
-    NVFP4_CUDA_TRY(cudaGetLastError());
+    const int64_t nb_pad = pad_to(p.k / 16, 4);
+    if (p.sf_rows_end == 0) return NVFP4_OK;
+    // One thread per (row, 16-element block); launches of at most 2^30 threads
+    // keep the in-kernel index 32-bit.
+    const int64_t rows_per_launch = ((int64_t)1 << 30) / nb_pad;
+    if (rows_per_launch < 1) return fail(NVFP4_ERR_UNSUPPORTED, "quantise: k too large");
+    for (int64_t r0 = 0; r0 < p.sf_rows_end; r0 += rows_per_launch) {
+        const int64_t rows = p.sf_rows_end - r0 < rows_per_launch ? p.sf_rows_end - r0 : rows_per_launch;
+        QuantLaunch l;
+        l.row_begin = r0;
+        l.nb_pad = (uint32_t)nb_pad;
+        l.total = (uint32_t)(rows * nb_pad);
+        const unsigned blocks = (unsigned)((l.total + kQuantThreads - 1) / kQuantThreads);
+        quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, l);
+        NVFP4_CUDA_TRY(cudaGetLastError());
+    }
     return NVFP4_OK;
 }
 
@@ -360,7 +389,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     if (m >= (1ll << 31) || n >= (1ll << 31) || k >= (1ll << 31))
         return fail(NVFP4_ERR_UNSUPPORTED, "gemm: dimension >= 2^31");
     if (odt != NVFP4_OUT_BF16 && odt != NVFP4_OUT_FP32) return fail(NVFP4_ERR_INVALID_ARG, "gemm: bad output dtype");
-    if (flags > NVFP4_GEMM_FORCE_DECODE) return fail(NVFP4_ERR_INVALID_ARG, "gemm: unknown flags 0x%x", flags);
+    if (flags > NVFP4_GEMM_FORCE_LARGE_PAIR) return fail(NVFP4_ERR_INVALID_ARG, "gemm: unknown flags 0x%x", flags);
     if (ldc < n) return fail(NVFP4_ERR_INVALID_ARG, "gemm: ldc %lld < n %lld", (long long)ldc, (long long)n);
     SegTable table;
     nvfp4_status st = check_segments(segs, nsegs, n, &table);
@@ -398,7 +427,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     p.splits = 1;
 
     CUtensorMap ta, tw;
-    if (!use_decode) {
+    if (!use_decode && flags != NVFP4_GEMM_FORCE_LARGE_PAIR) {
         p.m_tiles = (int)((m + large::BM - 1) / large::BM);
         p.n_tiles = (int)((n + large::BN - 1) / large::BN);
         if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
@@ -407,6 +436,32 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
         gemm_large_kernel<<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, p);
         NVFP4_CUDA_TRY(cudaGetLastError());
+        return ok();
+    }
+    if (!use_decode) {
+        // NVFP4_GEMM_FORCE_LARGE_PAIR: CTA pairs, 256 x 256 tiles, one pair per two SMs.
+        p.m_tiles = (int)((m + 255) / 256);
+        p.n_tiles = (int)((n + pairk::BN - 1) / pairk::BN);
+        CUtensorMap tsa, tsw;
+        if ((st = encode_fp4_map(&ta, a_q, m, k, pairk::CTA_ROWS)) != NVFP4_OK) return st;
+        if ((st = encode_fp4_map(&tw, w_q, n, k, pairk::BN / 2)) != NVFP4_OK) return st;
+        if ((st = encode_sf_map(&tsa, a_sf, m, k, 1)) != NVFP4_OK) return st;
+        if ((st = encode_sf_map(&tsw, w_sf, n, k, 2)) != NVFP4_OK) return st;
+        const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+        const int pairs = (int)(tiles < dev->sms / 2 ? tiles : dev->sms / 2);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+        cfg.blockDim = dim3(pairk::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = pairk::SMEM_BYTES;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tw, tsa, tsw, p));
         return ok();
     }
 

@@ -104,27 +104,48 @@ __device__ __forceinline__ float load_scale(const QuantParams& p)
 // integer atomicMax on the (non-negative) float bits: order-independent and
 // therefore deterministic.  *out must hold 0 (or a smaller amax) beforehand.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float absmax_vec(const void* base, int64_t elem_index, int in_fp32)
+{
+    if (in_fp32) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_index));
+        return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    }
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem_index));
+    // |bf16| as the float with the sign bit cleared; both halves of each word.
+    float m = 0.0f;
+    m = fmaxf(m, __uint_as_float((v.x << 16) & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float(v.x & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float((v.y << 16) & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float(v.y & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float((v.z << 16) & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float(v.z & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float((v.w << 16) & 0x7FFF0000u));
+    m = fmaxf(m, __uint_as_float(v.w & 0x7FFF0000u));
+    return m;
+}
+
 __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, int64_t rows, int64_t cols,
                                                    int64_t ldx, int in_fp32, unsigned int* __restrict__ out)
 {
-    const int64_t vec = in_fp32 ? 4 : 8;  // elements per 16-byte load
-    const int64_t vpr = cols / vec;       // cols % 32 == 0
-    const int64_t total = rows * vpr;
+    const int64_t vec = in_fp32 ? 4 : 8;  // elements per 16-byte load; cols % 32 == 0
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / vpr, c = (i - r * vpr) * vec;
-        if (in_fp32) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(x) + r * ldx + c));
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        } else {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + r * ldx + c));
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                m = fmaxf(m, fabsf(__uint_as_float(w[j] << 16)));
-                m = fmaxf(m, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
-            }
+    if (ldx == cols) {
+        // contiguous: one flat pass, four independent loads in flight per thread
+        const int64_t nvec = rows * cols / vec;
+        int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; i + 3 * stride < nvec; i += 4 * stride) {
+            const float a0 = absmax_vec(x, i * vec, in_fp32);
+            const float a1 = absmax_vec(x, (i + stride) * vec, in_fp32);
+            const float a2 = absmax_vec(x, (i + 2 * stride) * vec, in_fp32);
+            const float a3 = absmax_vec(x, (i + 3 * stride) * vec, in_fp32);
+            m = fmaxf(m, fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)));
         }
+        for (; i < nvec; i += stride) m = fmaxf(m, absmax_vec(x, i * vec, in_fp32));
+    } else {
+        for (int64_t r = blockIdx.x; r < rows; r += gridDim.x)
+            for (int64_t c = (int64_t)threadIdx.x * vec; c < cols; c += (int64_t)blockDim.x * vec)
+                m = fmaxf(m, absmax_vec(x, r * ldx + c, in_fp32));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -139,101 +160,96 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, i
 }
 
 // ---------------------------------------------------------------------------
-// Block quantiser.  A warp handles one 256-element segment of one row per
-// unit (8 elements per lane, two lanes per 16-element block) and UNITS
-// consecutive units per pass, issuing all loads first.
+// Block quantiser: one thread per 16-element block.  Threads are numbered
+// row-major over rows [row_begin, row_begin + grid rows) x the padded block
+// columns [0, 4 * katoms), so a warp reads 32 consecutive blocks (512 values)
+// of a row and writes 256 consecutive packed bytes.  Each group of four lanes
+// holds one 32-bit word of a scale atom, which its first lane stores.
+// Threads on padding (row >= rows or block >= K/16) write zero scales only.
 // ---------------------------------------------------------------------------
-constexpr int kQuantUnits = 4;
 constexpr int kQuantThreads = 256;
 
-__device__ __forceinline__ void load8(const QuantParams& p, int64_t r, int64_t c0, bool live, float (&v)[8])
+struct QuantLaunch {
+    int64_t row_begin;    // first (relative) row of this launch
+    uint32_t nb_pad;      // 4 * katoms
+    uint32_t total;       // threads that map to a (row, block): rows_in_launch * nb_pad
+};
+
+__device__ __forceinline__ void load16(const QuantParams& p, int64_t r, int64_t c0, float (&v)[16])
 {
-    if (!live) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-        return;
-    }
     if (p.in_fp32) {
-        const float* src = static_cast<const float*>(p.x) + r * p.ldx + c0;
-        const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(src + 4));
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-        const uint4 a = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r * p.ldx + c0));
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + r * p.ldx + c0);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            v[2 * j] = __uint_as_float(w[j] << 16);
-            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            const float4 a = __ldg(src + j);
+            v[4 * j] = a.x;
+            v[4 * j + 1] = a.y;
+            v[4 * j + 2] = a.z;
+            v[4 * j + 3] = a.w;
+        }
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r * p.ldx + c0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 a = __ldg(src + h);
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
+                v[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p)
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p,
+                                                               const QuantLaunch l)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t segs = (p.k + 255) / 256;
-    const int64_t nb = p.k / 16;
-    const int64_t katoms = (nb + 3) / 4;
-    const int64_t units = p.sf_rows_end * segs;
-    const int64_t warp_global = ((int64_t)blockIdx.x * kQuantThreads + threadIdx.x) >> 5;
-    const int64_t u0 = warp_global * kQuantUnits;
-    if (u0 >= units) return;
+    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
+    const uint32_t lane = threadIdx.x & 31u;
+    const bool mapped = t < l.total;
+    const uint32_t rl = mapped ? t / l.nb_pad : 0u;
+    const uint32_t kb = mapped ? t - rl * l.nb_pad : 0u;
+    const int64_t r = l.row_begin + rl;
+    const int64_t nb = p.k >> 4;
+    const bool live = mapped && r < p.rows && (int64_t)kb < nb;
 
     const float s_g = load_scale(p);
-    if (p.scale_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.scale_out = s_g;
-    const float t6 = __fmul_rn(6.0f, s_g);
+    if (p.scale_out != nullptr && t == 0 && l.row_begin == 0) *p.scale_out = s_g;
 
-    float v[kQuantUnits][8];
+    float v[16];
+    if (live) {
+        load16(p, r, (int64_t)kb * 16, v);
+    } else {
 #pragma unroll
-    for (int u = 0; u < kQuantUnits; ++u) {
-        const int64_t unit = u0 + u;
-        const int64_t r = unit / segs, seg = unit - r * segs;
-        const int64_t c0 = seg * 256 + lane * 8;
-        const bool live = unit < units && r < p.rows && c0 < p.k;
-        load8(p, r, c0, live, v[u]);
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
     }
-
+    float bm = 0.0f;
 #pragma unroll
-    for (int u = 0; u < kQuantUnits; ++u) {
-        const int64_t unit = u0 + u;
-        if (unit >= units) break;  // warp-uniform
-        const int64_t r = unit / segs, seg = unit - r * segs;
-        const int64_t c0 = seg * 256 + lane * 8;
-        const bool row_live = r < p.rows;
-        const bool live = row_live && c0 < p.k;
-
-        float bm = 0.0f;
+    for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(v[j]));
+    const uint32_t sb = live ? float_to_e4m3(__fdiv_rn(bm, __fmul_rn(6.0f, s_g))) : 0u;
+    const float se = __fmul_rn(e4m3_to_float(sb), s_g);
+    uint2 packed = make_uint2(0u, 0u);
+    if (se != 0.0f) {
+        float inv = __frcp_rn(se);
+        if (inv > FLT_MAX) inv = FLT_MAX;
+        float y[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) bm = fmaxf(bm, fabsf(v[u][j]));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-
-        const uint32_t sb = live ? float_to_e4m3(__fdiv_rn(bm, t6)) : 0u;
-        const float se = __fmul_rn(e4m3_to_float(sb), s_g);
-        uint32_t packed = 0;
-        if (se != 0.0f) {
-            float inv = __frcp_rn(se);
-            if (inv > FLT_MAX) inv = FLT_MAX;
-            float y[8];
+        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[j], inv);
+        packed.x = float8_to_e2m1x8(y);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[u][j], inv);
-            packed = float8_to_e2m1x8(y);
-        }
-        const int64_t grow = p.row_offset + r;
-        if (live) *reinterpret_cast<uint32_t*>(p.q + grow * (p.k / 2) + c0 / 2) = packed;
+        for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[8 + j], inv);
+        packed.y = float8_to_e2m1x8(y);
+    }
+    const int64_t grow = p.row_offset + r;
+    if (live) *reinterpret_cast<uint2*>(p.q + grow * (p.k >> 1) + (int64_t)kb * 8) = packed;
 
-        // Scale bytes: even lanes own block kb = seg*16 + lane/2.  Gather each
-        // group of four consecutive blocks (one 32-bit word of an atom row) in
-        // lane 8i and store it whole; blocks past K/16 contribute zero padding.
-        const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
-        const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 4);
-        const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 6);
-        const int64_t kb0 = seg * 16 + (lane >> 1);
-        if ((lane & 7) == 0 && kb0 < katoms * 4) {
-            const uint32_t word = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
-            *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb0, katoms)) = word;
-        }
+    const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
+    const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
+    const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
+    if (mapped && (lane & 3u) == 0u) {
+        const uint32_t word = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb, l.nb_pad >> 2)) = word;
     }
 }
 

@@ -20,6 +20,7 @@ from helpers import (act_from_codes, assert_gemm_close, dequant_codes, gemm_chec
 
 pytestmark = pytest.mark.gpu
 LARGE, DECODE, AUTO = nv.NVFP4_GEMM_FORCE_LARGE, nv.NVFP4_GEMM_FORCE_DECODE, nv.NVFP4_GEMM_AUTO
+PAIR = nv.NVFP4_GEMM_FORCE_LARGE_PAIR
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -35,12 +36,12 @@ def _w_hat_segments(codes, sf, segments):
 
 # --------------------------------------------------------------------------- constructed operands
 @pytest.mark.parametrize("kind", ["unit_scales", "row_scales", "kblock_scales", "random"])
-@pytest.mark.parametrize("flags", [LARGE, DECODE])
+@pytest.mark.parametrize("flags", [LARGE, DECODE, PAIR])
 def test_gemm_constructed_operands(kind, flags):
     """Operands built directly from codes and scale bytes isolate the data path
     (unit scales), the scale row mapping and the scale K mapping."""
     rng = np.random.default_rng({"unit_scales": 1, "row_scales": 2, "kblock_scales": 3, "random": 4}[kind])
-    m = 48 if flags == DECODE else 200
+    m = 48 if flags == DECODE else 300
     n, k = 384, 512
     ca = rng.integers(0, 16, (m, k)).astype(np.uint8)
     cw = rng.integers(0, 16, (n, k)).astype(np.uint8)
@@ -85,7 +86,7 @@ def _oracle_linear(p, rows=None):
     return c64, info["a_hat"], oracle.fused_weight_hat(info["qmods"])
 
 
-@pytest.mark.parametrize("flags", [AUTO, LARGE])
+@pytest.mark.parametrize("flags", [AUTO, LARGE, PAIR])
 def test_config_tiny_fp32_and_bf16(flags):
     """64x256 FP32 activations with one x50 column against a 128x256 FP32 weight."""
     p = synthetic.tiny()
@@ -112,7 +113,7 @@ RAGGED = [
 
 
 @pytest.mark.parametrize("m,widths,k", RAGGED)
-@pytest.mark.parametrize("flags", [AUTO, LARGE])
+@pytest.mark.parametrize("flags", [AUTO, LARGE, PAIR])
 def test_gemm_ragged_shapes_and_mid_tile_segments(m, widths, k, flags):
     a, _ = synthetic.activations(m, k, seed=m + k)
     stds = [0.02 if i % 2 == 0 else 0.2 for i in range(len(widths))]
@@ -147,7 +148,7 @@ def test_fused_segments_equal_unfused_modules_and_shared_scale_fails():
         assert ratio > 1.0 and fro > 2e-3, (shared, ratio, fro)
 
 
-@pytest.mark.parametrize("flags", [LARGE, DECODE])
+@pytest.mark.parametrize("flags", [LARGE, DECODE, PAIR])
 def test_gemm_is_deterministic(flags):
     m = 40 if flags == DECODE else 300
     p = synthetic.gdn_in_proj(m=m, k=1024, widths=(512, 48, 48, 1024), stds=(0.02, 0.2, 0.2, 0.02))
