@@ -97,7 +97,8 @@ __device__ __forceinline__ void store8(void* c, int64_t ldc, int out_fp32, int r
 //   0      TMA producer: A/B tiles and the stage's scale atoms into a 4-stage ring
 //   1      MMA issuer: tcgen05 block-scaled MMAs (M=128, N=256, K=64)
 //   2      owns the TMEM allocation
-//   4..11  epilogue: drain the accumulator, scale by s_ga * s_gw[segment], store
+//   4..11  epilogue: drain the accumulator, scale by s_ga * s_gw[segment],
+//          convert and store 16 x 32 chunks through shared memory with TMA
 //   12..15 scale staging: read each stage's scale atoms from shared memory and
 //          write them into TMEM with tcgen05.st (one warp per 32-lane quadrant,
 //          every quadrant receiving the full atom), keeping the tensor pipe free
@@ -152,7 +153,9 @@ constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int OFF_C = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int C_WARP = 1024;                       // per epilogue warp: one 16 x 32 BF16 chunk
+constexpr int OFF_BAR = OFF_C + 8 * C_WARP;
 // full[S], empty[S], sf_ready[2], sf_free[2], acc_full[2], acc_empty[2], ovl_free, drain
 constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 2 + 1 + 1;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
@@ -163,11 +166,12 @@ constexpr int ACC1_COL = 160;                         // ACC0 at 0; overlap [160
 constexpr int SF_COL = 416;                           // two scale slots of 48 columns
 constexpr int SF_SLOT = 48;                           // 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
 static_assert(ACC1_COL + BN <= SF_COL && SF_COL + 2 * SF_SLOT <= TMEM_COLS, "TMEM budget");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace large
 
 __global__ void __launch_bounds__(large::THREADS, 1)
     gemm_large_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ GemmParams p)
+                      const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ GemmParams p)
 {
     using namespace large;
     extern __shared__ uint8_t smem_raw[];
@@ -189,6 +193,7 @@ __global__ void __launch_bounds__(large::THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensor_map(&tmap_a);
         prefetch_tensor_map(&tmap_w);
+        prefetch_tensor_map(&tmap_c);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -398,18 +403,32 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
-                if (row < p.m) {
-                    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
+                // Store through this warp's 1 KB buffer: 16 rows x 32 BF16 columns
+                // (64-byte rows in the 64-byte swizzle the C tensor map uses); the
+                // copy engine clips rows and columns past the matrix.
+                uint8_t* cbuf = smem + OFF_C + ew * C_WARP;
+                const int row0 = mb * BM + quad * 32;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < 4; ++j) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int col = ncol0 + j * 32 + g * 8;
-                            if (col < p.n)
-                                *reinterpret_cast<uint4*>(crow + col) =
-                                    make_uint4(packed[j][4 * g], packed[j][4 * g + 1], packed[j][4 * g + 2],
-                                               packed[j][4 * g + 3]);
+                    for (int hr = 0; hr < 2; ++hr) {
+                        if (lane == 0) bulk_wait_group_read<0>();
+                        __syncwarp();
+                        if ((lane >> 4) == hr) {
+                            const int r = lane & 15;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                *reinterpret_cast<uint4*>(cbuf + r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) =
+                                    make_uint4(packed[j][4 * u], packed[j][4 * u + 1], packed[j][4 * u + 2],
+                                               packed[j][4 * u + 3]);
                         }
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0 && row0 + 16 * hr < p.m && ncol0 + j * 32 < p.n) {
+                            tma_store_2d(&tmap_c, cbuf, ncol0 + j * 32, row0 + 16 * hr);
+                            bulk_commit_group();
+                        }
+                    }
                 }
             } else {
                 for (int jj = 0; jj < 4; ++jj) {
@@ -446,6 +465,10 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         }
     }
 
+    if (warp >= 4 && warp < 12) {
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {

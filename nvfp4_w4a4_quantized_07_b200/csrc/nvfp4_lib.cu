@@ -118,6 +118,25 @@ nvfp4_status encode_fp4_map(CUtensorMap* map, const uint8_t* base, int64_t rows,
     return NVFP4_OK;
 }
 
+// Output C (m x n, row stride ldc elements) for TMA stores of 32-column
+// chunks from swizzled shared memory: BF16 chunks are 16 rows of 64 bytes
+// (64-byte swizzle); the FP32 map (32 x 32, 128-byte swizzle) is encoded for
+// completeness, FP32 output is written with plain stores.  Stores past m or n
+// are clipped by the copy engine.
+nvfp4_status encode_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64_t ldc, bool fp32)
+{
+    const cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)m};
+    const cuuint64_t strides[1] = {(cuuint64_t)(ldc * (fp32 ? 4 : 2))};
+    const cuuint32_t box[2] = {32u, fp32 ? 32u : 16u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          fp32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
 // Tiled scale buffer viewed as 32-bit words: dim 0 = the 128 words of one
 // 512-byte atom, dim 1 = K-atoms, dim 2 = 128-row blocks.  A box of
 // {128, 4, box_blocks} is one pipeline stage's scales; atoms past the end of
@@ -432,9 +451,11 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         p.n_tiles = (int)((n + large::BN - 1) / large::BN);
         if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
         if ((st = encode_fp4_map(&tw, w_q, n, k, large::BN)) != NVFP4_OK) return st;
+        CUtensorMap tc;
+        if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
-        gemm_large_kernel<<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, p);
+        gemm_large_kernel<<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tc, p);
         NVFP4_CUDA_TRY(cudaGetLastError());
         return ok();
     }
