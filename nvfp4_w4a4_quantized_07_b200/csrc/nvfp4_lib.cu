@@ -191,20 +191,34 @@ nvfp4_status launch_amax(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t
     return NVFP4_OK;
 }
 
+// Multiply-shift constants for exact unsigned division by d (1 <= d < 2^31) of
+// every dividend t < 2^30:  t / d == umulhi(4 t, mul) >> shift  with
+// shift = ceil(log2 d) and mul = ceil(2^(30 + shift) / d) (< 2^32).  The
+// rounding error t (mul - 2^(30+shift)/d) / 2^(30+shift) stays below
+// 2^-shift <= 1/d, so the floor is exact.
+void magic_divider(uint32_t d, uint32_t* mul, uint32_t* shift)
+{
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    *mul = (uint32_t)(((1ull << (30 + s)) + d - 1) / d);
+    *shift = s;
+}
+
 nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s)
 {
-    const int64_t nb_pad = pad_to(p.k / 16, 4);
+    const int64_t pairs = pad_to(p.k / 16, 4) / 2;
     if (p.sf_rows_end == 0) return NVFP4_OK;
-    // One thread per (row, 16-element block); launches of at most 2^30 threads
-    // keep the in-kernel index 32-bit.
-    const int64_t rows_per_launch = ((int64_t)1 << 30) / nb_pad;
+    // One thread per (row, pair of 16-element blocks); launches of at most
+    // 2^30 threads keep the in-kernel index 32-bit.
+    const int64_t rows_per_launch = ((int64_t)1 << 30) / pairs;
     if (rows_per_launch < 1) return fail(NVFP4_ERR_UNSUPPORTED, "quantise: k too large");
+    QuantLaunch l;
+    l.pairs = (uint32_t)pairs;
+    magic_divider(l.pairs, &l.div_mul, &l.div_shift);
     for (int64_t r0 = 0; r0 < p.sf_rows_end; r0 += rows_per_launch) {
         const int64_t rows = p.sf_rows_end - r0 < rows_per_launch ? p.sf_rows_end - r0 : rows_per_launch;
-        QuantLaunch l;
         l.row_begin = r0;
-        l.nb_pad = (uint32_t)nb_pad;
-        l.total = (uint32_t)(rows * nb_pad);
+        l.total = (uint32_t)(rows * pairs);
         const unsigned blocks = (unsigned)((l.total + kQuantThreads - 1) / kQuantThreads);
         quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, l);
         NVFP4_CUDA_TRY(cudaGetLastError());

@@ -160,76 +160,33 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, i
 }
 
 // ---------------------------------------------------------------------------
-// Block quantiser: one thread per 16-element block.  Threads are numbered
-// row-major over rows [row_begin, row_begin + grid rows) x the padded block
-// columns [0, 4 * katoms), so a warp reads 32 consecutive blocks (512 values)
-// of a row and writes 256 consecutive packed bytes.  Each group of four lanes
-// holds one 32-bit word of a scale atom, which its first lane stores.
-// Threads on padding (row >= rows or block >= K/16) write zero scales only.
+// Block quantiser: one thread per two consecutive 16-element blocks.  Threads
+// are numbered row-major over rows [row_begin, row_begin + launch rows) x the
+// padded block pairs [0, 2 * katoms), so a warp reads 64 consecutive blocks
+// (1024 values) of a row and writes 512 consecutive packed bytes.  Two
+// neighbouring lanes hold one 32-bit word of a scale atom (four blocks), which
+// the even lane stores.  Threads on padding (row >= rows or block >= K/16)
+// write zero scales only.
 // ---------------------------------------------------------------------------
 constexpr int kQuantThreads = 256;
 
 struct QuantLaunch {
     int64_t row_begin;    // first (relative) row of this launch
-    uint32_t nb_pad;      // 4 * katoms
-    uint32_t total;       // threads that map to a (row, block): rows_in_launch * nb_pad
+    uint32_t pairs;       // block pairs per row: 2 * katoms
+    uint32_t total;       // threads that map to a (row, pair): rows_in_launch * pairs
+    uint32_t div_mul;     // t / pairs == __umulhi(4 t, div_mul) >> div_shift for t < 2^30
+    uint32_t div_shift;
 };
 
-__device__ __forceinline__ void load16(const QuantParams& p, int64_t r, int64_t c0, float (&v)[16])
+__device__ __forceinline__ void quantize_block16(const float (&v)[16], float s_g, bool live, uint32_t& sb,
+                                                 uint2& packed)
 {
-    if (p.in_fp32) {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + r * p.ldx + c0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 a = __ldg(src + j);
-            v[4 * j] = a.x;
-            v[4 * j + 1] = a.y;
-            v[4 * j + 2] = a.z;
-            v[4 * j + 3] = a.w;
-        }
-    } else {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r * p.ldx + c0);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint4 a = __ldg(src + h);
-            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
-                v[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-            }
-        }
-    }
-}
-
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p,
-                                                               const QuantLaunch l)
-{
-    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
-    const uint32_t lane = threadIdx.x & 31u;
-    const bool mapped = t < l.total;
-    const uint32_t rl = mapped ? t / l.nb_pad : 0u;
-    const uint32_t kb = mapped ? t - rl * l.nb_pad : 0u;
-    const int64_t r = l.row_begin + rl;
-    const int64_t nb = p.k >> 4;
-    const bool live = mapped && r < p.rows && (int64_t)kb < nb;
-
-    const float s_g = load_scale(p);
-    if (p.scale_out != nullptr && t == 0 && l.row_begin == 0) *p.scale_out = s_g;
-
-    float v[16];
-    if (live) {
-        load16(p, r, (int64_t)kb * 16, v);
-    } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-    }
     float bm = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) bm = fmaxf(bm, fabsf(v[j]));
-    const uint32_t sb = live ? float_to_e4m3(__fdiv_rn(bm, __fmul_rn(6.0f, s_g))) : 0u;
+    sb = live ? float_to_e4m3(__fdiv_rn(bm, __fmul_rn(6.0f, s_g))) : 0u;
     const float se = __fmul_rn(e4m3_to_float(sb), s_g);
-    uint2 packed = make_uint2(0u, 0u);
+    packed = make_uint2(0u, 0u);
     if (se != 0.0f) {
         float inv = __frcp_rn(se);
         if (inv > FLT_MAX) inv = FLT_MAX;
@@ -241,15 +198,78 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_co
         for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(v[8 + j], inv);
         packed.y = float8_to_e2m1x8(y);
     }
-    const int64_t grow = p.row_offset + r;
-    if (live) *reinterpret_cast<uint2*>(p.q + grow * (p.k >> 1) + (int64_t)kb * 8) = packed;
+}
 
-    const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 1);
-    const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 2);
-    const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 3);
-    if (mapped && (lane & 3u) == 0u) {
-        const uint32_t word = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb, l.nb_pad >> 2)) = word;
+__device__ __forceinline__ void unpack_bf16x8(const uint4& a, float* v)
+{
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+}
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p,
+                                                               const QuantLaunch l)
+{
+    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
+    const uint32_t lane = threadIdx.x & 31u;
+    const bool mapped = t < l.total;
+    const uint32_t rl = mapped ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
+    const uint32_t pr = mapped ? t - rl * l.pairs : 0u;
+    const int64_t r = l.row_begin + rl;
+    const int64_t nb = p.k >> 4;
+    const int64_t kb0 = (int64_t)pr * 2;
+    const bool row_live = mapped && r < p.rows;
+    const bool live0 = row_live && kb0 < nb;
+    const bool live1 = row_live && kb0 + 1 < nb;
+
+    const float s_g = load_scale(p);
+    if (p.scale_out != nullptr && t == 0 && l.row_begin == 0) *p.scale_out = s_g;
+
+    // Issue every load of both blocks before any arithmetic.
+    float v0[16], v1[16];
+    if (p.in_fp32) {
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + r * p.ldx + kb0 * 16);
+        float4 f[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            f[j] = ((j < 4) ? live0 : live1) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v0[4 * j] = f[j].x; v0[4 * j + 1] = f[j].y; v0[4 * j + 2] = f[j].z; v0[4 * j + 3] = f[j].w;
+            v1[4 * j] = f[4 + j].x; v1[4 * j + 1] = f[4 + j].y; v1[4 * j + 2] = f[4 + j].z; v1[4 * j + 3] = f[4 + j].w;
+        }
+    } else {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r * p.ldx + kb0 * 16);
+        uint4 u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = ((j < 2) ? live0 : live1) ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+        unpack_bf16x8(u[0], v0);
+        unpack_bf16x8(u[1], v0 + 8);
+        unpack_bf16x8(u[2], v1);
+        unpack_bf16x8(u[3], v1 + 8);
+    }
+
+    uint32_t sb0, sb1;
+    uint2 q0, q1;
+    quantize_block16(v0, s_g, live0, sb0, q0);
+    quantize_block16(v1, s_g, live1, sb1, q1);
+    const int64_t grow = p.row_offset + r;
+    uint8_t* qdst = p.q + grow * (p.k >> 1) + kb0 * 8;
+    if (live1)
+        *reinterpret_cast<uint4*>(qdst) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    else if (live0)
+        *reinterpret_cast<uint2*>(qdst) = q0;
+
+    // Four consecutive blocks form one 32-bit word of an atom row.
+    const uint32_t half = sb0 | (sb1 << 8);
+    const uint32_t other = __shfl_down_sync(0xffffffffu, half, 1);
+    if (mapped && (pr & 1u) == 0u) {
+        const uint32_t word = half | (other << 16);
+        *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb0, l.pairs >> 1)) = word;
     }
 }
 
