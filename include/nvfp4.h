@@ -102,8 +102,10 @@ NVFP4_API int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k);
  * compute the global scale themselves (an amax accumulator). */
 NVFP4_API size_t nvfp4_quant_workspace_size(void);
 
-/* Workspace bytes nvfp4_gemm needs (currently 0 for every shape: the split-K
- * reduction runs through distributed shared memory). */
+/* Workspace bytes nvfp4_gemm needs for this shape and kernel choice: 0 for
+ * the large-M kernels; for the decode kernel (m <= 64) per-CTA flags plus one
+ * FP32 partial tile per CTA (at most ~8.4 MB).  The workspace needs no
+ * initialisation, but two calls that may run concurrently must not share one. */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags);
 
 /* ------------------------------------------------------------------------
@@ -171,8 +173,11 @@ NVFP4_API nvfp4_status nvfp4_quantize_act(const void* a, nvfp4_in_dtype dt, int6
  *                     multiple of 16, scales positive and finite.
  *   c, odt, ldc       device output, m x n, BF16 or FP32, row stride ldc
  *                     elements (ldc >= n, 16-byte aligned rows).
- *   workspace         device, >= nvfp4_gemm_workspace_size(...) bytes (may be
- *                     NULL when that is 0).
+ *   workspace         device, >= nvfp4_gemm_workspace_size(m, n, k, flags)
+ *                     bytes, 16-byte aligned (may be NULL when that is 0).
+ *                     The decode kernel passes partial tiles between its CTAs
+ *                     through it; it is launched cooperatively (all CTAs
+ *                     resident), one CTA per SM.
  *   flags             NVFP4_GEMM_* kernel choice.
  * Shapes: m >= 1, n a multiple of 16, k a multiple of 32, all < 2^31.
  * The BF16 output is the round-to-nearest-even BF16 of the FP32 output of the

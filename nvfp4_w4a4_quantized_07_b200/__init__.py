@@ -207,10 +207,28 @@ def segment_array(segments):
     return arr
 
 
+_ws_cache = {}
+
+
+def gemm_workspace(m: int, n: int, k: int, flags: int, device):
+    """A cached per-device workspace of at least nvfp4_gemm_workspace_size bytes."""
+    import torch
+    need = int(load().nvfp4_gemm_workspace_size(m, n, k, flags))
+    if need == 0:
+        return None
+    key = torch.device(device)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=key)
+        _ws_cache[key] = ws
+    return ws
+
+
 def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NVFP4_GEMM_AUTO,
-         segments=None, out=None):
+         segments=None, out=None, workspace=None):
     """``C = nvfp4_gemm(a, w)``: m x n output, BF16 by default.  ``segments``
-    overrides the fused weight's own segment table."""
+    overrides the fused weight's own segment table; ``workspace`` defaults to a
+    cached per-device buffer when the chosen kernel needs one."""
     import torch
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     if a.k != w.k:
@@ -221,9 +239,12 @@ def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NV
     odt = {torch.bfloat16: NVFP4_OUT_BF16, torch.float32: NVFP4_OUT_FP32}[out.dtype]
     arr = segment_array(segments)
     L = load()
+    if workspace is None:
+        workspace = gemm_workspace(a.m, w.n, w.k, flags, out.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("nvfp4_gemm", L.nvfp4_gemm(
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
-        _ptr(out), odt, out.stride(0), None, 0, flags, _stream(out.device)))
+        _ptr(out), odt, out.stride(0), _ptr(workspace), ws_bytes, flags, _stream(out.device)))
     return out
 
 

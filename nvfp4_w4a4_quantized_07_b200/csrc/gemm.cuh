@@ -20,10 +20,11 @@
 //    (M=128, N=256, K=64 per instruction) into a TMEM accumulator, warp 2 owns
 //    the TMEM allocation, warps 4..11 drain the accumulator and apply the
 //    segment scales.
-//  * gemm_decode_kernel: small M (<= 64 tokens).  Swap-AB (128 weight rows
-//    fill the MMA's M, the tokens its N) and split-K over a thread-block
-//    cluster; the partial accumulators are summed in a fixed rank order through
-//    distributed shared memory, so the result is deterministic.
+//  * gemm_decode_kernel: small M (<= 64 tokens), bound by streaming the weight.
+//    Stream-K: the (256-column tile, 256-deep k-tile) units are split evenly
+//    over one CTA per SM; a tile whose k-range spans several CTAs is finished
+//    by the CTA holding its first k-tile, which adds the others' FP32 partials
+//    in CTA order, so the result is deterministic.
 #pragma once
 
 #include <cuda.h>
@@ -53,7 +54,12 @@ struct GemmParams {
     SegTable segs;
     int m_tiles, n_tiles, k_tiles, katoms;
     int a_rowblocks, w_rowblocks;
-    int splits;                 // decode kernel: K-splits (= cluster size)
+    int splits;                 // (unused by the current kernels)
+    // decode kernel (stream-K): work units = w_tiles x k_tiles, split evenly
+    // over `ctas` co-resident CTAs; partial tiles meet in `ws`
+    int units, ctas;
+    uint8_t* ws;                // [256] uint64 flags, then [256][BT][256] FP32 partial tiles
+    unsigned long long epoch;   // this call's flag value
 };
 
 __device__ __forceinline__ float segment_scale(const SegTable& t, int col)
@@ -730,71 +736,134 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
 }
 
 // ===========================================================================
-// Decode kernel: swap-AB, split-K over a cluster, DSMEM reduction.
+// Decode kernel (M <= 64): stream-K over 256-column output tiles.
+//
+// Small M is pure weight streaming, and on this hardware every TMA / bulk
+// copy instruction and every block-scaled MMA has a fixed issue cost (~150
+// cycles) whatever its size.  So the kernel keeps both large: the tokens are
+// the MMA's M side (a 128-row operand of which only the first M rows are
+// loaded and stored -- the rest is never read back), 256 weight rows its N
+// side, 32 KB weight tiles per stage.  The (256-column tile, 256-deep k-tile)
+// work units are split evenly over exactly one CTA per SM (a cooperative
+// launch keeps them all resident).  A tile whose k-tiles span several CTAs is
+// finished by the CTA holding its first k-tile: the others reach their part of
+// it first, leave FP32 partials in the workspace and publish them with this
+// call's epoch value; the owner adds them in CTA order, so the result does not
+// depend on timing.
+//
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocation, 4..7
+// epilogue (TMEM quadrants 0-3 = token rows 0..127), 8..11 scale staging.
+// TMEM: accumulator [0, 256), four 48-column scale slots [256, 448).
 // ===========================================================================
 namespace decode {
-constexpr int BW = 128;                      // weight rows per CTA (the MMA's M)
+constexpr int BN = 256;                      // output columns (weight rows) per tile = the MMA's N
 constexpr int BK_BYTES = 128;
 constexpr int KSTEPS = 4;
-constexpr int THREADS = 256;                 // 4 control warps + 4 epilogue warps
-constexpr int W_STAGE = BW * BK_BYTES;       // 16 KB
-constexpr int SF_STAGE = 4 * 512;            // 4 atoms (weights) / 4 atoms (tokens)
-constexpr int TMEM_SF_STAGE = 32;            // 16 (weights) + 16 (tokens)
+constexpr int THREADS = 384;
+constexpr int B_STAGE = BN * BK_BYTES;       // 32 KB of weights
+constexpr int SFA_STAGE = 4 * 512;           // token scale atoms (one 128-row block)
+constexpr int SFB_STAGE = 2 * 4 * 512;       // weight scale atoms (two 128-row blocks)
+constexpr int SF_SLOTS = 4;
+constexpr int ACC_PITCH = BN + 4;            // floats per staged accumulator row: float4 access is conflict-free
+constexpr int TMEM_COLS = 512;
+constexpr int SF_COL = 256;
+constexpr int SF_SLOT = 48;                  // 16 (tokens: 4 k-steps x 4) + 32 (weights: 4 x 8)
+constexpr int MAX_CTAS = 256;
+constexpr int FLAGS_BYTES = MAX_CTAS * 8;
+static_assert(SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "TMEM budget");
 
+// Shared-memory plan for BT token rows.  The A stage holds only the BT loaded
+// rows; the M = 128 MMA reads 16 KB from its start, running on into the next
+// buffers, and the accumulator rows that come from those bytes are never read.
 template <int BT>
-struct Layout {
+struct Cfg {
     static constexpr int STAGES = BT >= 64 ? 3 : 4;
-    static constexpr int T_STAGE = BT * BK_BYTES;
-    static constexpr int OFF_W = 0;
-    static constexpr int OFF_T = OFF_W + STAGES * W_STAGE;
-    static constexpr int OFF_SFW = OFF_T + STAGES * (T_STAGE < 1024 ? 1024 : T_STAGE);
-    static constexpr int OFF_SFT = OFF_SFW + STAGES * SF_STAGE;
-    static constexpr int OFF_BAR = OFF_SFT + STAGES * SF_STAGE;
-    static constexpr int NUM_BARS = 2 * STAGES + 1;
-    static constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;
-    static constexpr int RED_BYTES = BW * BT * 4;  // partial sums, reuses the operand ring
-    static constexpr int TMEM_COLS = 256;
-    static constexpr int TMEM_SF = BT;             // scale ring after the accumulator
-    static_assert(RED_BYTES <= OFF_BAR, "reduction buffer must fit in the operand ring");
-    static_assert(BT + STAGES * TMEM_SF_STAGE <= TMEM_COLS, "TMEM budget");
+    static constexpr int A_STAGE = BT * BK_BYTES;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+    static constexpr int OFF_ACC = OFF_SFB + STAGES * SFB_STAGE;
+    static constexpr int OFF_BAR = OFF_ACC + BT * ACC_PITCH * 4;
+    // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full, acc_empty, drain
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, acc_full verdict, peer-wait verdict
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static_assert(A_STAGE % 1024 == 0, "SW128 stages are 1 KB aligned");
+    static_assert(OFF_A + (STAGES - 1) * A_STAGE + 128 * BK_BYTES <= OFF_MISC, "MMA A reads stay in the buffer");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+// Which CTA's range holds unit u when `units` are split over `ctas`:
+// CTA c owns [floor(c U / G), floor((c+1) U / G)).
+__device__ __forceinline__ int cta_of_unit(int64_t u, int units, int ctas)
+{
+    return (int)(((u + 1) * ctas + units - 1) / units) - 1;
+}
 }  // namespace decode
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 template <int BT>
-__global__ void __launch_bounds__(decode::THREADS, 2)
+__global__ void __launch_bounds__(decode::THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ GemmParams p)
 {
     using namespace decode;
-    using L = Layout<BT>;
+    using C = Cfg<BT>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int A_STAGE = C::A_STAGE;
+    constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_SFA = C::OFF_SFA, OFF_SFB = C::OFF_SFB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
-    uint64_t* empty = full + L::STAGES;
-    uint64_t* tmem_full = empty + L::STAGES;
-    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM_PTR);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* sf_ready = empty + STAGES;
+    uint64_t* sf_free = sf_ready + SF_SLOTS;
+    uint64_t* acc_full = sf_free + SF_SLOTS;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* drain = acc_empty + 1;
+    uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* acc_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);    // acc_full verdict
+    volatile int* peers_bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8); // a peer wait ran out
+    float* acc_stage = reinterpret_cast<float*>(smem + C::OFF_ACC);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int wt = blockIdx.x;               // weight-row tile
-    const int split = blockIdx.y;            // K split = rank in the cluster
-    const int kt_per = (p.k_tiles + p.splits - 1) / p.splits;
-    const int kt0 = min(split * kt_per, p.k_tiles);
-    const int kt1 = min(kt0 + kt_per, p.k_tiles);
+    const int cta = blockIdx.x;
+    const int64_t u_begin = (int64_t)cta * p.units / p.ctas;
+    const int64_t u_end = (int64_t)(cta + 1) * p.units / p.ctas;
+    const int k_tiles = p.k_tiles;
 
     if (warp == 0 && lane == 0) {
         prefetch_tensor_map(&tmap_a);
         prefetch_tensor_map(&tmap_w);
-        for (int s = 0; s < L::STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tmem_full, 1);
+        for (int i = 0; i < SF_SLOTS; ++i) {
+            mbar_init(&sf_ready[i], 4);
+            mbar_init(&sf_free[i], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(drain, 1);
+        *peers_bad = 0;
         fence_mbarrier_init();
     }
     if (warp == 2) {
-        tmem_alloc(tmem_ptr, L::TMEM_COLS);
+        tmem_alloc(tmem_ptr, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -803,156 +872,305 @@ __global__ void __launch_bounds__(decode::THREADS, 2)
     const uint32_t tmem_base = *tmem_ptr;
 
     if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int issued = 0;
-            for (int kt = kt0; kt < kt1; ++kt) {
-                if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) break;
+            bool ok = true;
+            int nb = (int)(u_begin / k_tiles), kt = (int)(u_begin - (int64_t)nb * k_tiles);
+            for (int64_t u = u_begin; u < u_end; ++u) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
+                    ok = false;
+                    break;
+                }
                 const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
                 const uint32_t sf_bytes = (uint32_t)nks * 512u;
-                mbar_arrive_expect_tx(&full[stage], W_STAGE + L::T_STAGE + 2 * sf_bytes);
-                tma_load_2d(smem + L::OFF_W + stage * W_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, wt * BW);
-                tma_load_2d(smem + L::OFF_T + stage * (L::T_STAGE < 1024 ? 1024 : L::T_STAGE), &tmap_a, &full[stage],
-                            kt * BK_BYTES, 0);
-                bulk_load(smem + L::OFF_SFW + stage * SF_STAGE, p.w_sf + ((int64_t)wt * p.katoms + kt * KSTEPS) * 512,
-                          sf_bytes, &full[stage]);
-                bulk_load(smem + L::OFF_SFT + stage * SF_STAGE, p.a_sf + ((int64_t)kt * KSTEPS) * 512, sf_bytes,
+                const bool rb1 = 2 * nb + 1 < p.w_rowblocks;
+                mbar_arrive_expect_tx(&full[stage], BT * BK_BYTES + B_STAGE + sf_bytes * (rb1 ? 3u : 2u));
+                tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES, 0);
+                tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, nb * BN);
+                bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_sf + (int64_t)kt * KSTEPS * 512, sf_bytes,
                           &full[stage]);
-                ++issued;
-                if (++stage == L::STAGES) {
+                bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
+                          p.w_sf + ((int64_t)(2 * nb) * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
+                if (rb1)
+                    bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
+                              p.w_sf + ((int64_t)(2 * nb + 1) * p.katoms + kt * KSTEPS) * 512, sf_bytes,
+                              &full[stage]);
+                if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
+                if (++kt == k_tiles) {
+                    kt = 0;
+                    ++nb;
+                }
             }
-            (void)issued;
+            if (!ok) {
+                const long long t0 = clock64();
+                while (clock64() - t0 < kWaitCycles / 64) {
+                }
+            }
         }
         __syncwarp();
     } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = idesc_nvf4(BW, BT);
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int kt = kt0; kt < kt1; ++kt) {
-                if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull)) break;
+            const uint32_t idesc = idesc_nvf4(128, BN);
+            int stage = 0, slot = 0;
+            uint32_t slot_phase = 0, segs = 0;
+            bool ok = true, first = true;
+            int kt = (int)(u_begin % k_tiles);
+            for (int64_t u = u_begin; u < u_end && ok; ++u) {
+                if (u == u_begin || kt == 0) {
+                    // a new segment: the accumulator has been drained
+                    if (!mbar_wait(acc_empty, (segs & 1) ^ 1, kStatusTimeoutAccum)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    first = true;
+                }
+                if (!mbar_wait(&sf_ready[slot], slot_phase, kStatusTimeoutFull)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
-                const uint32_t sf_col = tmem_base + L::TMEM_SF + stage * TMEM_SF_STAGE;
-                const uint8_t* sfw = smem + L::OFF_SFW + stage * SF_STAGE;
-                const uint8_t* sft = smem + L::OFF_SFT + stage * SF_STAGE;
-                for (int ks = 0; ks < nks; ++ks) {
-                    tmem_cp_32x128b_x4(sf_col + 4 * ks, desc_sf_atom(sfw + ks * 512));
-                    tmem_cp_32x128b_x4(sf_col + 16 + 4 * ks, desc_sf_atom(sft + ks * 512));
-                }
-                const uint64_t wdesc = desc_kmajor_sw128(smem + L::OFF_W + stage * W_STAGE);
-                const uint64_t tdesc =
-                    desc_kmajor_sw128(smem + L::OFF_T + stage * (L::T_STAGE < 1024 ? 1024 : L::T_STAGE));
+                const uint32_t sf_col = tmem_base + SF_COL + slot * SF_SLOT;
+                const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
+                const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
                 for (int ks = 0; ks < nks; ++ks)
-                    mma_nvf4(tmem_base, wdesc + 2 * ks, tdesc + 2 * ks, idesc, (kt != kt0) || (ks != 0),
-                             sf_col + 4 * ks, sf_col + 16 + 4 * ks);
+                    mma_nvf4(tmem_base, adesc + 2 * ks, bdesc + 2 * ks, idesc, !(first && ks == 0), sf_col + 4 * ks,
+                             sf_col + 16 + 8 * ks);
+                first = false;
                 mma_commit(&empty[stage]);
-                if (++stage == L::STAGES) {
-                    stage = 0;
-                    phase ^= 1;
+                mma_commit(&sf_free[slot]);
+                if (++stage == STAGES) stage = 0;
+                if (++slot == SF_SLOTS) {
+                    slot = 0;
+                    slot_phase ^= 1;
                 }
+                if (u == u_end - 1 || kt == k_tiles - 1) {
+                    mma_commit(acc_full);
+                    ++segs;
+                }
+                if (++kt == k_tiles) kt = 0;
             }
-            mma_commit(tmem_full);
+            if (!ok) {
+                mma_commit(drain);
+                mbar_wait(drain, 0, kStatusTimeoutDrain, kWaitCycles / 8);
+            }
         }
         __syncwarp();
-    }
-
-    // ---------------------------------------------------------------- partials
-    // Epilogue warps 4..7: weight row = 32*(warp%4) + lane; BT token columns.
-    float* red = reinterpret_cast<float*>(smem);  // [BT][BW], reuses the operand ring
-    const bool have_k = kt1 > kt0;
-    if (warp >= 4) {
-        const int quad = warp & 3;
-        const int wrow = quad * 32 + lane;
-        bool ok = true;
-        if (have_k) ok = mbar_wait(tmem_full, 0, kStatusTimeoutAccum);
-        if (ok && have_k) tc_fence_after();
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ scale staging
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0, slot_phase = 0;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull) ||
+                !mbar_wait(&sf_free[slot], slot_phase ^ 1, kStatusTimeoutFull))
+                break;
+            tc_fence_after();
+            const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE + lane * 16;
+            const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE + lane * 16;
+            uint32_t ra[16], rb[16], rc[16];
 #pragma unroll
-        for (int c = 0; c < BT; c += 16) {
-            uint32_t v[16];
-            if (have_k && ok) {
-                tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(quad * 32) << 16) + c, v);
-                tmem_ld_wait();
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = 0u;
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint4 a = *reinterpret_cast<const uint4*>(sfa + ks * 512);
+                ra[4 * ks] = a.x;
+                ra[4 * ks + 1] = a.y;
+                ra[4 * ks + 2] = a.z;
+                ra[4 * ks + 3] = a.w;
+                const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + ks * 512);
+                const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + ks * 512);
+                uint32_t* d = ks < 2 ? rb : rc;
+                const int o = (ks & 1) * 8;
+                d[o] = b0.x;
+                d[o + 1] = b0.y;
+                d[o + 2] = b0.z;
+                d[o + 3] = b0.w;
+                d[o + 4] = b1.x;
+                d[o + 5] = b1.y;
+                d[o + 6] = b1.z;
+                d[o + 7] = b1.w;
             }
-            if (p.splits == 1) {
-                const int n = wt * BW + wrow;
-                if (n < p.n) {
-                    const float alpha = __fmul_rn(*p.act_scale, segment_scale(p.segs, n));
+            const uint32_t col = tmem_base + lane_base + SF_COL + slot * SF_SLOT;
+            tmem_st_32x32b_x16(col, ra);
+            tmem_st_32x32b_x16(col + 16, rb);
+            tmem_st_32x32b_x16(col + 32, rc);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sf_ready[slot]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+            if (++slot == SF_SLOTS) {
+                slot = 0;
+                slot_phase ^= 1;
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        // Per segment (one tile's k-range): the warps whose TMEM lanes hold
+        // token rows move the FP32 accumulator into shared memory and release
+        // TMEM at once, so the MMAs of the next segment start while this one is
+        // reduced and stored.  Then all 128 epilogue threads work on the staged
+        // tile, 4 consecutive columns of one row each: a contributor writes its
+        // partial to the workspace and publishes it; the owner adds the other
+        // CTAs' partials in CTA order, scales each column by s_ga * s_gw[seg]
+        // and stores the output.  Every branch below is uniform over the four
+        // warps, so the named barrier (id 1, 128 threads) always matches.
+        const int quad = warp & 3;
+        const int et = threadIdx.x - 128;          // 0..127
+        const int t = quad * 32 + lane;            // token row = accumulator lane
+        const bool live = quad * 32 < BT;          // warp holds loaded token rows
+        unsigned long long* flags = reinterpret_cast<unsigned long long*>(p.ws);
+        float* parts = reinterpret_cast<float*>(p.ws + FLAGS_BYTES);
+        const float s_ga = *p.act_scale;
+        constexpr int DU = 4;                      // float4 units per thread per pass
+    constexpr int PG = 4;                      // peers whose loads are in flight together
+    const int mrows = min(p.m, BT);
+        const int units4 = mrows * (BN / 4);       // float4 units of the live rows
+        uint32_t segs = 0;
+        int64_t u = u_begin;
+        while (u < u_end) {
+            const int nb = (int)(u / k_tiles), kb = (int)(u - (int64_t)nb * k_tiles);
+            const int64_t seg_end = min(u_end, (int64_t)(nb + 1) * k_tiles);
+            const bool owner = kb == 0;
+            const bool complete = owner && seg_end == (int64_t)(nb + 1) * k_tiles;
+            const int last = owner && !complete ? cta_of_unit((int64_t)(nb + 1) * k_tiles - 1, p.units, p.ctas) : cta;
+
+            if (et == 0) *acc_ok = mbar_wait(acc_full, segs & 1, kStatusTimeoutAccum) ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (!*acc_ok) break;
+            tc_fence_after();
+            if (live) {
+                const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+                float* row = acc_stage + t * ACC_PITCH;
+#pragma unroll 1
+                for (int j = 0; j < BN / 32; j += 2) {
+                    uint32_t r0[32], r1[32];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32(taddr + j * 32, r0);
+                    tmem_ld_32x32b_x32(taddr + (j + 1) * 32, r1);
+                    tmem_ld_wait();
+                    if (t < BT) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int t = c + e;
-                        if (t < p.m) {
-                            const float o = __fmul_rn(__uint_as_float(v[e]), alpha);
-                            if (p.out_fp32)
-                                static_cast<float*>(p.c)[(int64_t)t * p.ldc + n] = o;
-                            else
-                                static_cast<__nv_bfloat16*>(p.c)[(int64_t)t * p.ldc + n] = __float2bfloat16_rn(o);
+                        for (int e = 0; e < 32; e += 4) {
+                            *reinterpret_cast<float4*>(row + j * 32 + e) =
+                                make_float4(__uint_as_float(r0[e]), __uint_as_float(r0[e + 1]),
+                                            __uint_as_float(r0[e + 2]), __uint_as_float(r0[e + 3]));
+                            *reinterpret_cast<float4*>(row + (j + 1) * 32 + e) =
+                                make_float4(__uint_as_float(r1[e]), __uint_as_float(r1[e + 1]),
+                                            __uint_as_float(r1[e + 2]), __uint_as_float(r1[e + 3]));
                         }
                     }
                 }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) red[(c + e) * BW + wrow] = __uint_as_float(v[e]);
             }
-        }
-    }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            ++segs;
 
-    if (p.splits > 1) {
-        // All CTAs of the cluster hold their partials in shared memory now.
-        cluster_arrive_release();
-        cluster_wait_acquire();
-        // Rank r sums its slice of the BT x BW partial tile over ranks 0..S-1 in
-        // order, scales, converts and stores.
-        const uint32_t red_addr = smem_u32(red);
-        constexpr int kVec = BT * BW / 4;
-        const int per = (kVec + p.splits - 1) / p.splits;
-        const int v0 = split * per, v1 = min(v0 + per, kVec);
-        const float s_ga = *p.act_scale;
-        for (int i = v0 + (int)threadIdx.x; i < v1; i += THREADS) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int r = 0; r < p.splits; ++r) {
-                const float4 x = ld_shared_cluster_f4(map_shared_rank(red_addr + 16u * (uint32_t)i, (uint32_t)r));
-                acc.x = __fadd_rn(acc.x, x.x);
-                acc.y = __fadd_rn(acc.y, x.y);
-                acc.z = __fadd_rn(acc.z, x.z);
-                acc.w = __fadd_rn(acc.w, x.w);
-            }
-            const int t = (4 * i) / BW;
-            const int wrow = (4 * i) % BW;
-            const int n = wt * BW + wrow;
-            if (t < p.m && n < p.n) {
-                // n % 4 == 0 and n < p.n with p.n % 16 == 0: the 4 columns stay inside one 16-column group.
-                const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, n));
-                const float o0 = __fmul_rn(acc.x, alpha), o1 = __fmul_rn(acc.y, alpha);
-                const float o2 = __fmul_rn(acc.z, alpha), o3 = __fmul_rn(acc.w, alpha);
-                if (p.out_fp32) {
-                    *reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)t * p.ldc + n) =
-                        make_float4(o0, o1, o2, o3);
-                } else {
-                    uint2 w;
-                    w.x = pack_bf16x2(o0, o1);
-                    w.y = pack_bf16x2(o2, o3);
-                    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)t * p.ldc + n) = w;
+            if (owner && !complete) {
+                // thread i waits for CTAs cta + 1 + i, cta + 1 + i + 128, ... to
+                // publish their partials of tile nb
+                for (int i = et; i < last - cta; i += 128) {
+                    const long long t0 = clock64();
+                    while (ld_acquire_u64(flags + cta + 1 + i) != p.epoch) {
+                        if (clock64() - t0 > kWaitCycles) {
+                            record_status(kStatusTimeoutCluster);
+                            *peers_bad = 1;
+                            break;
+                        }
+                    }
                 }
             }
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // staged tile complete, peers acquired
+            if (*peers_bad) break;
+
+            if (!owner) {
+                float* mine = parts + (int64_t)cta * BT * BN;
+                for (int x = et; x < units4; x += 128) {
+                    const int r = x / (BN / 4), c4 = x % (BN / 4);
+                    __stcg(reinterpret_cast<float4*>(mine + r * BN) + c4,
+                           *reinterpret_cast<const float4*>(acc_stage + r * ACC_PITCH + 4 * c4));
+                }
+                __threadfence();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (et == 0) st_release_u64(flags + cta, p.epoch);
+            } else {
+                // DU units per thread at a time; the loads of PG peers are in
+                // flight together and added in CTA order.
+                for (int x0 = et; x0 < units4; x0 += DU * 128) {
+                    float4 v[DU];
+#pragma unroll
+                    for (int i = 0; i < DU; ++i) {
+                        const int x = x0 + i * 128;
+                        if (x < units4)
+                            v[i] = *reinterpret_cast<const float4*>(acc_stage + (x / (BN / 4)) * ACC_PITCH +
+                                                                    4 * (x % (BN / 4)));
+                    }
+                    for (int c2 = cta + 1; c2 <= last; c2 += PG) {
+                        float4 q[PG][DU];
+#pragma unroll
+                        for (int g = 0; g < PG; ++g) {
+                            const float* src = parts + (int64_t)(c2 + g) * BT * BN;
+#pragma unroll
+                            for (int i = 0; i < DU; ++i) {
+                                const int x = x0 + i * 128;
+                                if (x < units4 && c2 + g <= last)
+                                    q[g][i] = __ldcg(reinterpret_cast<const float4*>(
+                                        src + (x / (BN / 4)) * BN + 4 * (x % (BN / 4))));
+                            }
+                        }
+#pragma unroll
+                        for (int g = 0; g < PG; ++g) {
+                            if (c2 + g <= last) {
+#pragma unroll
+                                for (int i = 0; i < DU; ++i) {
+                                    v[i].x = __fadd_rn(v[i].x, q[g][i].x);
+                                    v[i].y = __fadd_rn(v[i].y, q[g][i].y);
+                                    v[i].z = __fadd_rn(v[i].z, q[g][i].z);
+                                    v[i].w = __fadd_rn(v[i].w, q[g][i].w);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < DU; ++i) {
+                        const int x = x0 + i * 128;
+                        const int r = x / (BN / 4);
+                        const int col = nb * BN + 4 * (x % (BN / 4));
+                        if (x < units4 && col < p.n) {
+                            // 4 columns never straddle a segment (boundaries are multiples of 16)
+                            const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
+                            const float o0 = __fmul_rn(v[i].x, alpha), o1 = __fmul_rn(v[i].y, alpha);
+                            const float o2 = __fmul_rn(v[i].z, alpha), o3 = __fmul_rn(v[i].w, alpha);
+                            if (p.out_fp32) {
+                                *reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)r * p.ldc + col) =
+                                    make_float4(o0, o1, o2, o3);
+                            } else {
+                                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)r * p.ldc +
+                                                          col) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+                            }
+                        }
+                    }
+                }
+            }
+            u = seg_end;
         }
-        // Nobody leaves while a peer may still read its shared memory.
-        cluster_arrive_release();
-        cluster_wait_acquire();
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, L::TMEM_COLS);
+        tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 

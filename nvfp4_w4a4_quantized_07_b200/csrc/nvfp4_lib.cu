@@ -9,7 +9,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
+#include <chrono>
 #include <mutex>
+#include <random>
 
 #include "../../include/nvfp4.h"
 #include "gemm.cuh"
@@ -79,11 +82,11 @@ nvfp4_status device_state(DeviceState** out)
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             pairk::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Layout<16>::SMEM_BYTES));
+                                            decode::Cfg<16>::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Layout<32>::SMEM_BYTES));
+                                            decode::Cfg<32>::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Layout<64>::SMEM_BYTES));
+                                            decode::Cfg<64>::SMEM_BYTES));
         d.ready = true;
     }
     *out = &d;
@@ -258,19 +261,44 @@ nvfp4_status check_segments(const nvfp4_segment* segs, int nsegs, int64_t n, Seg
     return NVFP4_OK;
 }
 
+// Bytes of workspace the decode kernel needs for m tokens: flags plus one FP32
+// partial tile per CTA.
+size_t decode_ws_bytes(int64_t m)
+{
+    const int64_t bt = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
+    return (size_t)decode::FLAGS_BYTES + (size_t)decode::MAX_CTAS * (size_t)bt * decode::BN * 4;
+}
+
+// Per-call flag values for the decode kernel's partial-tile hand-off: a random
+// 64-bit starting point (so values left in a reused workspace by another
+// process or an aborted call cannot match) advanced once per call.
+std::atomic<unsigned long long> g_epoch{0};
+std::once_flag g_epoch_once;
+
+unsigned long long next_epoch()
+{
+    std::call_once(g_epoch_once, [] {
+        std::random_device rd;
+        const unsigned long long seed = ((unsigned long long)rd() << 32) ^ rd() ^
+                                        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+        g_epoch.store(seed | 1ull);
+    });
+    return g_epoch.fetch_add(2ull) + 2ull;
+}
+
 template <int BT>
-nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, GemmParams p, int w_tiles, cudaStream_t s)
+nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& p, cudaStream_t s)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)w_tiles, (unsigned)p.splits, 1);
+    cfg.gridDim = dim3((unsigned)p.ctas, 1, 1);
     cfg.blockDim = dim3(decode::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = decode::Layout<BT>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = decode::Cfg<BT>::SMEM_BYTES;
     cfg.stream = s;
+    // The owners of split row tiles wait for the other CTAs' partials, so all
+    // CTAs must be resident at once.
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = (unsigned)p.splits;
-    attr[0].val.clusterDim.z = 1;
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT>, ta, tw, p));
@@ -299,7 +327,13 @@ int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k)
 
 size_t nvfp4_quant_workspace_size(void) { return 256; }
 
-size_t nvfp4_gemm_workspace_size(int64_t, int64_t, int64_t, uint32_t) { return 0; }
+size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags)
+{
+    (void)n;
+    (void)k;
+    const bool decode_path = flags == NVFP4_GEMM_FORCE_DECODE || (flags == NVFP4_GEMM_AUTO && m <= 64);
+    return decode_path && m >= 0 && m <= 64 ? decode_ws_bytes(m) : 0;
+}
 
 const char* nvfp4_get_last_error_string(void) { return g_err; }
 
@@ -414,8 +448,6 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
                         void* c, nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, uint32_t flags,
                         void* stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (m < 0 || n <= 0 || k <= 0 || n % 16 != 0 || k % 32 != 0)
         return fail(NVFP4_ERR_INVALID_ARG, "gemm: need m >= 0, n a positive multiple of 16, k a positive multiple of 32 "
                                            "(m=%lld n=%lld k=%lld)", (long long)m, (long long)n, (long long)k);
@@ -437,6 +469,12 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     const bool use_decode = flags == NVFP4_GEMM_FORCE_DECODE || (flags == NVFP4_GEMM_AUTO && m <= 64);
     if (use_decode && m > 64) return fail(NVFP4_ERR_UNSUPPORTED, "gemm: the decode kernel handles m <= 64");
     if (m == 0) return ok();
+    if (use_decode) {
+        if (workspace == nullptr || ws_bytes < decode_ws_bytes(m))
+            return fail(NVFP4_ERR_WORKSPACE, "gemm: the decode kernel needs %zu bytes of workspace (got %zu)",
+                        decode_ws_bytes(m), ws_bytes);
+        if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "gemm: workspace not 16-byte aligned");
+    }
 
     DeviceState* dev = nullptr;
     if ((st = device_state(&dev)) != NVFP4_OK) return st;
@@ -501,19 +539,22 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     }
 
     const int bt = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
-    const int w_tiles = (int)((n + decode::BW - 1) / decode::BW);
-    int splits = (2 * dev->sms) / w_tiles;
-    if (splits > 8) splits = 8;
-    if (splits > p.k_tiles) splits = p.k_tiles;
-    if (splits < 1) splits = 1;
-    p.splits = splits;
+    const int w_tiles = (int)((n + decode::BN - 1) / decode::BN);
+    const int64_t units = (int64_t)w_tiles * p.k_tiles;
+    if (units >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "gemm: decode problem too large");
+    int64_t ctas = dev->sms < decode::MAX_CTAS ? dev->sms : decode::MAX_CTAS;
+    if (ctas > units) ctas = units;
+    p.units = (int)units;
+    p.ctas = (int)ctas;
+    p.ws = static_cast<uint8_t*>(workspace);
+    p.epoch = next_epoch();
     p.m_tiles = 1;
     p.n_tiles = w_tiles;
     if ((st = encode_fp4_map(&ta, a_q, m, k, bt)) != NVFP4_OK) return st;
-    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BW)) != NVFP4_OK) return st;
-    if (bt == 16) st = launch_decode<16>(ta, tw, p, w_tiles, s);
-    else if (bt == 32) st = launch_decode<32>(ta, tw, p, w_tiles, s);
-    else st = launch_decode<64>(ta, tw, p, w_tiles, s);
+    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
+    if (bt == 16) st = launch_decode<16>(ta, tw, p, s);
+    else if (bt == 32) st = launch_decode<32>(ta, tw, p, s);
+    else st = launch_decode<64>(ta, tw, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
 }

@@ -146,6 +146,21 @@ def test_valid_call_without_a_gpu_fails_loudly(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     s = _segs((0, 64, 1.0))
-    st = lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None)
+    st = lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 200, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None)
     assert st in (2, 4)
     assert lib.nvfp4_get_last_error_string()
+    ws = ctypes.c_void_p(0x40000)
+    st = lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, ws, 1 << 24, 0, None)
+    assert st in (2, 4)
+
+
+def test_decode_gemm_requires_workspace(lib):
+    s = _segs((0, 64, 1.0))
+    need = lib.nvfp4_gemm_workspace_size(8, 64, 64, 0)
+    assert need > 0 and lib.nvfp4_gemm_workspace_size(8, 64, 64, 1) == 0
+    assert lib.nvfp4_gemm_workspace_size(300, 64, 64, 0) == 0
+    assert lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, None, 0, 0, None) == 6
+    ws = ctypes.c_void_p(0x40000)
+    assert lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, ws, need - 16, 0, None) == 6
+    assert lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, MISALIGNED, need, 0,
+                          None) == 3
