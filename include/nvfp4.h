@@ -103,8 +103,9 @@ NVFP4_API int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k);
 NVFP4_API size_t nvfp4_quant_workspace_size(void);
 
 /* Workspace bytes nvfp4_gemm needs for this shape and kernel choice: 0 for
- * the large-M kernels; for the decode kernel (m <= 64) per-CTA flags plus one
- * FP32 partial tile per CTA (at most ~8.4 MB).  The workspace needs no
+ * the large-M kernels; for the decode kernel (m <= 64) 2 KiB of per-CTA flags
+ * plus one 256-column FP32 partial tile of 16, 32 or 64 rows per CTA slot
+ * (256 slots): 4, 8 or 16 MiB.  The workspace needs no
  * initialisation, but two calls that may run concurrently must not share one. */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags);
 
