@@ -190,6 +190,43 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_gemm_decode_noalloc - the decode GEMM (the kernel nvfp4_gemm runs
+ * under NVFP4_GEMM_FORCE_DECODE) with no workspace argument.  The pages have
+ * no counterpart to this call; it exists for deployment.
+ *
+ * It is for callers that have no way to hand the library device scratch
+ * memory: an operator slot or plug-in interface with a fixed signature, or a
+ * plain C host with no device allocator; and for callers that must not
+ * allocate in the middle of a step, because a device allocation can block
+ * until the device is idle or fail when memory is tight.  The call allocates
+ * nothing.  The kernel's scratch (one flag per CTA slot and one FP32 partial
+ * tile per CTA slot) lives in a fixed array of NVFP4_NOALLOC_SCRATCH_BYTES
+ * bytes of device memory that the library reserves on each device it is
+ * loaded on.
+ *
+ * Arguments: as nvfp4_gemm without workspace, ws_bytes and flags.
+ * Limit: m <= NVFP4_NOALLOC_MAX_M tokens.  A larger m needs more scratch than
+ *   the array holds; the call then returns NVFP4_ERR_UNSUPPORTED and does
+ *   nothing (use nvfp4_gemm with a workspace).  m == 0 is a no-op.  Other
+ *   argument errors are those of nvfp4_gemm.
+ * Set-up: the first call on a device, made with that device current, looks up
+ *   the array's device address and sets the kernels' attributes.  Make that
+ *   first call before any stream capture begins.
+ * Sharing: every call on a device uses the same array.  Nothing in it has to
+ *   be zero when a call starts: a CTA's flag is compared with a value fresh to
+ *   each call, and every partial tile is written before it is read in the
+ *   same call.  Two calls that overlap in time on one device (different
+ *   streams, or threads without ordering) race on the array and give wrong
+ *   results; order them (one stream, or events).
+ * ---------------------------------------------------------------------- */
+#define NVFP4_NOALLOC_MAX_M 16
+#define NVFP4_NOALLOC_SCRATCH_BYTES (2048 + 256 * 16 * 256 * 4) /* 4 MiB + 2 KiB */
+NVFP4_API nvfp4_status nvfp4_gemm_decode_noalloc(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
+                                       const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t n, int64_t k,
+                                       const nvfp4_segment* segs, int nsegs, void* c, nvfp4_out_dtype odt,
+                                       int64_t ldc, void* stream);
+
+/* ------------------------------------------------------------------------
  * Diagnostics.
  * ---------------------------------------------------------------------- */
 

@@ -27,8 +27,10 @@ NVFP4_MAX_SEGMENTS = 16
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA", 5: "TIMEOUT",
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
-            "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_get_last_error_string",
-            "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout", "nvfp4_version")
+            "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_decode_noalloc",
+            "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
+            "nvfp4_version")
+NVFP4_NOALLOC_MAX_M = 16
 
 
 class NVFP4Error(RuntimeError):
@@ -67,6 +69,9 @@ def load():
     L.nvfp4_quantize_act.restype = INT
     L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
     L.nvfp4_gemm.restype = INT
+    L.nvfp4_gemm_decode_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64,
+                                            P]
+    L.nvfp4_gemm_decode_noalloc.restype = INT
     L.nvfp4_get_last_error_string.argtypes = []
     L.nvfp4_get_last_error_string.restype = ctypes.c_char_p
     L.nvfp4_check_device_status.argtypes = [P]
@@ -245,6 +250,21 @@ def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NV
     _check("nvfp4_gemm", L.nvfp4_gemm(
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
         _ptr(out), odt, out.stride(0), _ptr(workspace), ws_bytes, flags, _stream(out.device)))
+    return out
+
+
+def gemm_decode_noalloc(a: QuantizedActivation, w: FusedWeight, out, segments=None):
+    """``nvfp4_gemm_decode_noalloc``: the decode GEMM into the caller's ``out``
+    (m x n, BF16 or FP32) using the library's built-in scratch; neither this
+    wrapper nor the C call allocates device memory.  m <= 16."""
+    if a.k != w.k:
+        raise ValueError("K mismatch between activations and weight")
+    segments = w.segments if segments is None else segments
+    odt = NVFP4_OUT_FP32 if out.element_size() == 4 else NVFP4_OUT_BF16
+    arr = segment_array(segments)
+    _check("nvfp4_gemm_decode_noalloc", load().nvfp4_gemm_decode_noalloc(
+        _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
+        _ptr(out), odt, out.stride(0), _stream(out.device)))
     return out
 
 

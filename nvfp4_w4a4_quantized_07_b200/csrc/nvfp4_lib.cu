@@ -307,6 +307,40 @@ nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, const G
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Built-in scratch of nvfp4_gemm_decode_noalloc: the decode kernel's flags and
+// partial tiles for up to NVFP4_NOALLOC_MAX_M tokens and 256 CTA slots, in
+// device memory reserved when the module is loaded on a device (no allocation
+// call).  Its address on each device is looked up once, with that device
+// current.
+// ---------------------------------------------------------------------------
+static_assert(NVFP4_NOALLOC_SCRATCH_BYTES ==
+                  decode::FLAGS_BYTES + (size_t)decode::MAX_CTAS * NVFP4_NOALLOC_MAX_M * decode::BN * 4,
+              "scratch = flags + one 16-row partial tile per CTA slot");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+nvfp4_status noalloc_scratch(void** out)
+{
+    int dev = 0;
+    NVFP4_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        NVFP4_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+        if (ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 255u) != 0)
+            return fail(NVFP4_ERR_CUDA, "gemm_decode_noalloc: scratch address %p is not 256-byte aligned", ptr);
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return NVFP4_OK;
+}
+}  // namespace
+
 // ===========================================================================
 // C ABI
 // ===========================================================================
@@ -557,6 +591,28 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     else st = launch_decode<64>(ta, tw, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
+}
+
+nvfp4_status nvfp4_gemm_decode_noalloc(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
+                                       const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t n, int64_t k,
+                                       const nvfp4_segment* segs, int nsegs, void* c, nvfp4_out_dtype odt,
+                                       int64_t ldc, void* stream)
+{
+    if (m < 0) return fail(NVFP4_ERR_INVALID_ARG, "gemm_decode_noalloc: m = %lld < 0", (long long)m);
+    if (m > NVFP4_NOALLOC_MAX_M)
+        return fail(NVFP4_ERR_UNSUPPORTED,
+                    "gemm_decode_noalloc: m = %lld needs %zu bytes of decode scratch, but the built-in array holds "
+                    "%zu (m <= %d); call nvfp4_gemm with a workspace instead",
+                    (long long)m, decode_ws_bytes(m), (size_t)NVFP4_NOALLOC_SCRATCH_BYTES, NVFP4_NOALLOC_MAX_M);
+    void* scratch = nullptr;
+    if (m > 0) {
+        DeviceState* dev = nullptr;
+        nvfp4_status st = device_state(&dev);
+        if (st != NVFP4_OK) return st;
+        if ((st = noalloc_scratch(&scratch)) != NVFP4_OK) return st;
+    }
+    return nvfp4_gemm(a_q, a_sf, act_scale_dev, w_q, w_sf, m, n, k, segs, nsegs, c, odt, ldc, scratch,
+                      NVFP4_NOALLOC_SCRATCH_BYTES, NVFP4_GEMM_FORCE_DECODE, stream);
 }
 
 nvfp4_status nvfp4_check_device_status(void* stream)

@@ -164,3 +164,19 @@ def test_decode_gemm_requires_workspace(lib):
     assert lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, ws, need - 16, 0, None) == 6
     assert lib.nvfp4_gemm(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, s, 1, FAKE, 0, 64, MISALIGNED, need, 0,
                           None) == 3
+
+
+def test_decode_noalloc_limits_without_a_device(lib):
+    """The allocation-free decode call refuses m above its built-in scratch
+    before touching a device, and m == 0 is a no-op."""
+    s = _segs((0, 64, 1.0))
+    f = lib.nvfp4_gemm_decode_noalloc
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 17, 64, 64, s, 1, FAKE, 0, 64, None) == 2
+    msg = lib.nvfp4_get_last_error_string()
+    assert b"m <= 16" in msg and b"workspace" in msg
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 64, 64, s, 1, FAKE, 0, 64, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 64, 64, s, 1, FAKE, 0, 64, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 64, s, 1, FAKE, 0, 64, None) == 0
+    assert nv.NVFP4_NOALLOC_MAX_M == 16
+    # the built-in scratch is exactly the decode workspace for 16 tokens
+    assert lib.nvfp4_gemm_workspace_size(16, 64, 64, nv.NVFP4_GEMM_FORCE_DECODE) == 2048 + 256 * 16 * 256 * 4
