@@ -68,24 +68,31 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the GEMM kernel's device source (the counters of a profile hold
+    only for the source they were taken on)."""
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "ptx.cuh", "quant.cuh", "nvfp4_lib.cu"):
+    for f in ("gemm.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_07_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic():
-    """DRAM bytes per launch of the GEMM from the committed ncu summary, if it
-    was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "gemm_large_gdn_in_proj_8192.json")
+    """DRAM bytes per launch of the GEMM from the committed ncu summary
+    (``source_hash:`` and ``dram_bytes_per_launch:`` lines), if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "gemm_large_gdn_in_proj_8192.md")
     if not os.path.exists(path):
         return None
+    fields = {}
     with open(path) as f:
-        d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+        for line in f:
+            key, sep, val = line.strip().strip("`").partition(":")
+            if sep and key in ("source_hash", "dram_bytes_per_launch"):
+                fields[key] = val.strip().strip("`")
+    if fields.get("source_hash") != kernel_source_hash() or "dram_bytes_per_launch" not in fields:
         return None
-    return d.get("dram_bytes_per_launch")
+    return int(float(fields["dram_bytes_per_launch"]))
 
 
 # --------------------------------------------------------------------------- clocks
