@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--m", type=int, default=8192)
     ap.add_argument("--no-decode", action="store_true", help="skip the decode GB/s sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mlp", action="store_true", help="skip the prefill and long-prefill MLP measurements")
     ap.add_argument("--profile-gemm", action="store_true",
                     help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
     ap.add_argument("--decode-case", default=None,
@@ -414,7 +415,90 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
             del fwd
         out["decode"] = {"unit": "GB/s", "bytes": "W_q + W_sf + A_q + A_sf + C (bf16), L2 flushed",
                          "shapes": dec}
+    if not args.no_mlp:
+        out.update(prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks))
     return out
+
+
+def _timed(fn, flush, stream, device, reps=5, warm=2):
+    """Median CUDA-event time (ms) of ``fn`` after ``warm`` runs, L2 flushed before each."""
+    import torch
+    for _ in range(warm):
+        fn()
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        torch.cuda._sleep(1_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
+    """The other large-M workloads: a 4096x5120x5120 prefill projection and the
+    32768-token MLP (fused gate/up GEMM -> silu-mul glue with a dynamic scale ->
+    down GEMM), each timed as one whole step with inputs resident."""
+    import torch
+    res = {}
+    # ---- prefill: act quant (static scale) + GEMM
+    p = synthetic.prefill()
+    a = p.a.to(device)
+    fw = nv.quantize_weight([w.to(device) for w in p.modules])
+    s_a = nv.quantize_act(a).scale.clone()
+    aq = nv.quantize_act(a, act_scale=s_a)
+    c = torch.empty((p.m, p.n), dtype=torch.bfloat16, device=device)
+
+    def prefill_step():
+        nv.quantize_act(a, act_scale=s_a, out=aq)
+        nv.gemm(aq, fw, out=c)
+
+    ms = _timed(prefill_step, flush, stream, device)
+    flops = 2.0 * p.m * p.n * p.k
+    res["prefill_4096x5120x5120"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms}
+    del a, fw, aq, c
+
+    # ---- long-prefill MLP
+    p = synthetic.mlp_gate_up()
+    f = synthetic.MLP_INTERMEDIATE
+    a = p.a.to(device)
+    fw1 = nv.quantize_weight([w.to(device) for w in p.modules])
+    fw2 = nv.quantize_weight([synthetic.mlp_down_weight().to(device)])
+    s_a = nv.quantize_act(a).scale.clone()
+    aq = nv.quantize_act(a, act_scale=s_a)
+    c1 = torch.empty((p.m, 2 * f), dtype=torch.bfloat16, device=device)
+    c2 = torch.empty((p.m, p.k), dtype=torch.bfloat16, device=device)
+    ws = nv.quant_workspace(device)
+    hq = nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws)[0]
+
+    def stage(i):
+        if i == 0:
+            nv.quantize_act(a, act_scale=s_a, out=aq)
+        elif i == 1:
+            nv.gemm(aq, fw1, out=c1)
+        elif i == 2:
+            nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws, out=hq)
+        else:
+            nv.gemm(hq, fw2, out=c2)
+
+    def mlp_step():
+        for i in range(4):
+            stage(i)
+
+    ms = _timed(mlp_step, flush, stream, device, reps=3, warm=1)
+    flops = 2.0 * p.m * (2 * f) * p.k + 2.0 * p.m * p.k * f
+    glue_ms = _timed(lambda: stage(2), flush, stream, device, reps=3, warm=1)
+    glue_bytes = p.m * f * (2 * 2 * 2 + 0.5 + 1 / 16)      # g, u read twice (dynamic), codes + scales written
+    res["mlp_32768x5120_17408"] = {
+        "value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+        "gemm_gate_up_ms": _timed(lambda: stage(1), flush, stream, device, reps=3, warm=1),
+        "gemm_down_ms": _timed(lambda: stage(3), flush, stream, device, reps=3, warm=1),
+        "glue_ms": glue_ms, "glue_GB/s": glue_bytes / (glue_ms * 1e-3) / 1e9,
+        "glue_frac_hbm": glue_bytes / (glue_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    return res
 
 
 def run_decode_case(args):

@@ -190,6 +190,36 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_silu_mul_quantize - the glue of a gated (SwiGLU) MLP whose gate/up
+ * and down projections both run as W4A4 NVFP4 GEMMs: from the BF16 gate g and
+ * up u halves of the fused gate/up GEMM output it forms
+ *     h = bf16( silu(g) * u ),  silu(x) = x / (1 + e^-x)
+ * (every step in FP32 with round-to-nearest; e^-x is CUDA's expf, within 2
+ * ulp) and quantises h to NVFP4 exactly as nvfp4_quantize_act quantises an
+ * activation (the down projection's on-the-fly input quantisation).  The
+ * pages do not describe the MLP; this is the step between its two linear
+ * layers.
+ *
+ *   g, u              device BF16, m x f each, row stride ldgu elements
+ *                     (for a fused [gate | up] output of width 2f: g = C,
+ *                     u = C + f, ldgu = 2f); 16-byte aligned rows.
+ *   h_scale_dev       device FP32 decode scale of h (static), or NULL:
+ *                     dynamic, amax(h)/2688 computed on the device first.
+ *   h_scale_out_dev   device float receiving the scale used (required in
+ *                     dynamic mode).
+ *   h_q, h_sf         device outputs as for nvfp4_quantize_act with k = f.
+ *   h_out, ldh        optional device BF16 m x f copy of h (NULL: not
+ *                     written), row stride ldh.
+ *   workspace         device, >= nvfp4_quant_workspace_size() bytes, needed
+ *                     only in dynamic mode.
+ * Shapes: m >= 0, f a positive multiple of 32, both < 2^31.
+ * Dynamic mode reads g and u twice (amax pass, then the quantising pass).
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int64_t m, int64_t f, int64_t ldgu,
+                                     const float* h_scale_dev, float* h_scale_out_dev, uint8_t* h_q, uint8_t* h_sf,
+                                     void* h_out, int64_t ldh, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_gemm_decode_noalloc - the decode GEMM (the kernel nvfp4_gemm runs
  * under NVFP4_GEMM_FORCE_DECODE) with no workspace argument.  The pages have
  * no counterpart to this call; it exists for deployment.

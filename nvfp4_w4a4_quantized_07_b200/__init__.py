@@ -27,7 +27,8 @@ NVFP4_MAX_SEGMENTS = 16
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA", 5: "TIMEOUT",
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
-            "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_decode_noalloc",
+            "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
+            "nvfp4_gemm_decode_noalloc",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
 NVFP4_NOALLOC_MAX_M = 16
@@ -67,6 +68,8 @@ def load():
     L.nvfp4_quantize_weight.restype = INT
     L.nvfp4_quantize_act.argtypes = [P, INT, I64, I64, I64, P, P, P, P, P, SZ, P]
     L.nvfp4_quantize_act.restype = INT
+    L.nvfp4_silu_mul_quantize.argtypes = [P, P, I64, I64, I64, P, P, P, P, P, I64, P, SZ, P]
+    L.nvfp4_silu_mul_quantize.restype = INT
     L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
     L.nvfp4_gemm.restype = INT
     L.nvfp4_gemm_decode_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64,
@@ -168,6 +171,36 @@ def quantize_act(a, act_scale=None, workspace=None, out: QuantizedActivation | N
         _ptr(a), _in_dtype(a), m, k, a.stride(0), _ptr(act_scale), _ptr(out.scale), _ptr(out.q), _ptr(out.sf),
         _ptr(workspace), ws_bytes, _stream(a.device)))
     return out
+
+
+def silu_mul_quantize(g, u, h_scale=None, return_h: bool = False, workspace=None,
+                      out: QuantizedActivation | None = None):
+    """MLP glue (``nvfp4_silu_mul_quantize``): h = bf16(silu(g) * u) quantised
+    to NVFP4.  ``g`` and ``u`` are BF16 m x f CUDA tensors with unit column
+    stride and the same row stride (e.g. the two halves of a fused gate/up
+    GEMM output).  ``h_scale`` is a static 1-element FP32 device scale or
+    ``None`` (dynamic).  Returns ``(QuantizedActivation, h or None)``."""
+    import torch
+    _require_cuda(g, u, h_scale)
+    if g.dtype != torch.bfloat16 or u.dtype != torch.bfloat16:
+        raise TypeError("g and u must be bfloat16")
+    if g.shape != u.shape or g.dim() != 2 or g.stride() != u.stride() or g.stride(1) != 1:
+        raise ValueError("g and u must be 2-D tensors of one shape and row stride, unit column stride")
+    m, f = g.shape
+    L = load()
+    if out is None:
+        out = QuantizedActivation(
+            q=torch.empty((m, f // 2), dtype=torch.uint8, device=g.device),
+            sf=torch.empty(max(L.nvfp4_sf_bytes(m, f), 1), dtype=torch.uint8, device=g.device),
+            scale=torch.empty(1, dtype=torch.float32, device=g.device), m=m, k=f)
+    h = torch.empty((m, f), dtype=torch.bfloat16, device=g.device) if return_h else None
+    if h_scale is None and workspace is None:
+        workspace = quant_workspace(g.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("nvfp4_silu_mul_quantize", L.nvfp4_silu_mul_quantize(
+        _ptr(g), _ptr(u), m, f, g.stride(0), _ptr(h_scale), _ptr(out.scale), _ptr(out.q), _ptr(out.sf),
+        _ptr(h), f, _ptr(workspace), ws_bytes, _stream(g.device)))
+    return out, h
 
 
 def quantize_weight(modules, global_scales=None, workspace=None) -> FusedWeight:

@@ -814,6 +814,20 @@ __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned l
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Scale 4 consecutive output columns of one row by s_ga * s_gw[seg] and store
+// them (4 columns never straddle a segment: boundaries are multiples of 16).
+__device__ __forceinline__ void store4_scaled(const GemmParams& p, int row, int col, float s_ga, float4 v)
+{
+    const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
+    const float o0 = __fmul_rn(v.x, alpha), o1 = __fmul_rn(v.y, alpha);
+    const float o2 = __fmul_rn(v.z, alpha), o3 = __fmul_rn(v.w, alpha);
+    if (p.out_fp32)
+        *reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + col) = make_float4(o0, o1, o2, o3);
+    else
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col) =
+            make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+}
+
 template <int BT>
 __global__ void __launch_bounds__(decode::THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
@@ -860,6 +874,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         mbar_init(acc_empty, 4);
         mbar_init(drain, 1);
         *peers_bad = 0;
+        *acc_ok = 0;
         fence_mbarrier_init();
     }
     if (warp == 2) {
@@ -1018,12 +1033,14 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         // Per segment (one tile's k-range): the warps whose TMEM lanes hold
         // token rows move the FP32 accumulator into shared memory and release
         // TMEM at once, so the MMAs of the next segment start while this one is
-        // reduced and stored.  Then all 128 epilogue threads work on the staged
-        // tile, 4 consecutive columns of one row each: a contributor writes its
-        // partial to the workspace and publishes it; the owner adds the other
-        // CTAs' partials in CTA order, scales each column by s_ga * s_gw[seg]
-        // and stores the output.  Every branch below is uniform over the four
-        // warps, so the named barrier (id 1, 128 threads) always matches.
+        // stored.  Then all 128 epilogue threads work on the staged tile, 4
+        // consecutive columns of one row each: a contributor (a range that
+        // starts inside the tile) writes its partial to the workspace and
+        // publishes it; the owner of a tile that lies wholly in this range
+        // scales each column by s_ga * s_gw[seg] and stores the output.  An
+        // owner whose range ends inside the tile waits for the peers' flags and
+        // hands over to the all-warp finish below.  Every branch is uniform over
+        // the four warps, so the named barrier (id 1, 128 threads) always matches.
         const int quad = warp & 3;
         const int et = threadIdx.x - 128;          // 0..127
         const int t = quad * 32 + lane;            // token row = accumulator lane
@@ -1031,10 +1048,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         unsigned long long* flags = reinterpret_cast<unsigned long long*>(p.ws);
         float* parts = reinterpret_cast<float*>(p.ws + FLAGS_BYTES);
         const float s_ga = *p.act_scale;
-        constexpr int DU = 4;                      // float4 units per thread per pass
-    constexpr int PG = 4;                      // peers whose loads are in flight together
-    const int mrows = min(p.m, BT);
-        const int units4 = mrows * (BN / 4);       // float4 units of the live rows
+        const int units4 = min(p.m, BT) * (BN / 4);  // float4 units of the live rows
         uint32_t segs = 0;
         int64_t u = u_begin;
         while (u < u_end) {
@@ -1090,7 +1104,10 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                     }
                 }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");   // staged tile complete, peers acquired
+            // An owner whose range ends inside tile nb (always the CTA's last
+            // segment) leaves the reduction to all twelve warps, below.
+            if (owner && !complete) break;
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // staged tile complete
             if (*peers_bad) break;
 
             if (!owner) {
@@ -1104,35 +1121,64 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                 asm volatile("bar.sync 1, 128;" ::: "memory");
                 if (et == 0) st_release_u64(flags + cta, p.epoch);
             } else {
-                // DU units per thread at a time; the loads of PG peers are in
-                // flight together and added in CTA order.
-                for (int x0 = et; x0 < units4; x0 += DU * 128) {
-                    float4 v[DU];
+                // a complete tile: scale and store
+                for (int x = et; x < units4; x += 128) {
+                    const int r = x / (BN / 4);
+                    const int col = nb * BN + 4 * (x % (BN / 4));
+                    if (col < p.n)
+                        store4_scaled(p, r, col, s_ga,
+                                      *reinterpret_cast<const float4*>(acc_stage + r * ACC_PITCH + 4 * (x % (BN / 4))));
+                }
+            }
+            u = seg_end;
+        }
+    }
+
+    // ---------------------------------------------------------------- split-tile finish
+    // The CTA whose range starts tile nb = (u_end - 1) / k_tiles but ends inside
+    // it owns that tile's result: once the epilogue has staged this CTA's
+    // accumulator and acquired the peers' flags, all 384 threads add the peers'
+    // FP32 partials in CTA order (loads for FPG peers in flight together),
+    // scale and store.  The condition is the same for every thread.
+    {
+        const int64_t fin_nb = u_end > u_begin ? (u_end - 1) / k_tiles : 0;
+        const bool finish = u_end > u_begin && u_end % k_tiles != 0 && fin_nb * k_tiles >= u_begin;
+        if (finish) {
+            asm volatile("bar.sync 2, 384;" ::: "memory");
+            if (*acc_ok && !*peers_bad) {
+                constexpr int FDU = 3, FPG = 8;
+                const int nb = (int)fin_nb;
+                const int last = cta_of_unit((int64_t)(nb + 1) * k_tiles - 1, p.units, p.ctas);
+                const int units4 = min(p.m, BT) * (BN / 4);
+                const float* parts = reinterpret_cast<const float*>(p.ws + FLAGS_BYTES);
+                const float s_ga = *p.act_scale;
+                for (int x0 = threadIdx.x; x0 < units4; x0 += FDU * THREADS) {
+                    float4 v[FDU];
 #pragma unroll
-                    for (int i = 0; i < DU; ++i) {
-                        const int x = x0 + i * 128;
+                    for (int i = 0; i < FDU; ++i) {
+                        const int x = x0 + i * THREADS;
                         if (x < units4)
                             v[i] = *reinterpret_cast<const float4*>(acc_stage + (x / (BN / 4)) * ACC_PITCH +
                                                                     4 * (x % (BN / 4)));
                     }
-                    for (int c2 = cta + 1; c2 <= last; c2 += PG) {
-                        float4 q[PG][DU];
+                    for (int c2 = cta + 1; c2 <= last; c2 += FPG) {
+                        float4 q[FPG][FDU];
 #pragma unroll
-                        for (int g = 0; g < PG; ++g) {
+                        for (int g = 0; g < FPG; ++g) {
                             const float* src = parts + (int64_t)(c2 + g) * BT * BN;
 #pragma unroll
-                            for (int i = 0; i < DU; ++i) {
-                                const int x = x0 + i * 128;
+                            for (int i = 0; i < FDU; ++i) {
+                                const int x = x0 + i * THREADS;
                                 if (x < units4 && c2 + g <= last)
                                     q[g][i] = __ldcg(reinterpret_cast<const float4*>(
                                         src + (x / (BN / 4)) * BN + 4 * (x % (BN / 4))));
                             }
                         }
 #pragma unroll
-                        for (int g = 0; g < PG; ++g) {
+                        for (int g = 0; g < FPG; ++g) {
                             if (c2 + g <= last) {
 #pragma unroll
-                                for (int i = 0; i < DU; ++i) {
+                                for (int i = 0; i < FDU; ++i) {
                                     v[i].x = __fadd_rn(v[i].x, q[g][i].x);
                                     v[i].y = __fadd_rn(v[i].y, q[g][i].y);
                                     v[i].z = __fadd_rn(v[i].z, q[g][i].z);
@@ -1142,27 +1188,13 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                         }
                     }
 #pragma unroll
-                    for (int i = 0; i < DU; ++i) {
-                        const int x = x0 + i * 128;
-                        const int r = x / (BN / 4);
+                    for (int i = 0; i < FDU; ++i) {
+                        const int x = x0 + i * THREADS;
                         const int col = nb * BN + 4 * (x % (BN / 4));
-                        if (x < units4 && col < p.n) {
-                            // 4 columns never straddle a segment (boundaries are multiples of 16)
-                            const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col));
-                            const float o0 = __fmul_rn(v[i].x, alpha), o1 = __fmul_rn(v[i].y, alpha);
-                            const float o2 = __fmul_rn(v[i].z, alpha), o3 = __fmul_rn(v[i].w, alpha);
-                            if (p.out_fp32) {
-                                *reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)r * p.ldc + col) =
-                                    make_float4(o0, o1, o2, o3);
-                            } else {
-                                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)r * p.ldc +
-                                                          col) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
-                            }
-                        }
+                        if (x < units4 && col < p.n) store4_scaled(p, x / (BN / 4), col, s_ga, v[i]);
                     }
                 }
             }
-            u = seg_end;
         }
     }
 

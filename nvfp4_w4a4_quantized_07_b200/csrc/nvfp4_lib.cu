@@ -207,23 +207,32 @@ void magic_divider(uint32_t d, uint32_t* mul, uint32_t* shift)
     *shift = s;
 }
 
-nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s)
+enum QuantKind { kQuantPlain, kQuantSiluMul, kAmaxSiluMul };
+
+// One thread per (row, pair of 16-element blocks) over rows [0, rows_end);
+// launches of at most 2^30 threads keep the in-kernel index 32-bit.
+nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s, QuantKind kind = kQuantPlain,
+                          const SiluParams* sp = nullptr, unsigned int* amax = nullptr)
 {
     const int64_t pairs = pad_to(p.k / 16, 4) / 2;
-    if (p.sf_rows_end == 0) return NVFP4_OK;
-    // One thread per (row, pair of 16-element blocks); launches of at most
-    // 2^30 threads keep the in-kernel index 32-bit.
+    const int64_t rows_end = kind == kAmaxSiluMul ? p.rows : p.sf_rows_end;
+    if (rows_end == 0) return NVFP4_OK;
     const int64_t rows_per_launch = ((int64_t)1 << 30) / pairs;
     if (rows_per_launch < 1) return fail(NVFP4_ERR_UNSUPPORTED, "quantise: k too large");
     QuantLaunch l;
     l.pairs = (uint32_t)pairs;
     magic_divider(l.pairs, &l.div_mul, &l.div_shift);
-    for (int64_t r0 = 0; r0 < p.sf_rows_end; r0 += rows_per_launch) {
-        const int64_t rows = p.sf_rows_end - r0 < rows_per_launch ? p.sf_rows_end - r0 : rows_per_launch;
+    for (int64_t r0 = 0; r0 < rows_end; r0 += rows_per_launch) {
+        const int64_t rows = rows_end - r0 < rows_per_launch ? rows_end - r0 : rows_per_launch;
         l.row_begin = r0;
         l.total = (uint32_t)(rows * pairs);
         const unsigned blocks = (unsigned)((l.total + kQuantThreads - 1) / kQuantThreads);
-        quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, l);
+        if (kind == kQuantPlain)
+            quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, l);
+        else if (kind == kQuantSiluMul)
+            silu_mul_quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, *sp, l);
+        else
+            silu_mul_amax_kernel<<<blocks, kQuantThreads, 0, s>>>(p, *sp, l, amax);
         NVFP4_CUDA_TRY(cudaGetLastError());
     }
     return NVFP4_OK;
@@ -410,6 +419,65 @@ nvfp4_status nvfp4_quantize_act(const void* a, nvfp4_in_dtype dt, int64_t m, int
     p.scale_ptr = dynamic ? static_cast<const float*>(workspace) : act_scale_dev;
     p.scale_out = act_scale_out_dev;
     if ((st = launch_quant(p, s)) != NVFP4_OK) return st;
+    return ok();
+}
+
+nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int64_t m, int64_t f, int64_t ldgu,
+                                     const float* h_scale_dev, float* h_scale_out_dev, uint8_t* h_q, uint8_t* h_sf,
+                                     void* h_out, int64_t ldh, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (m < 0 || f <= 0 || f % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "silu_mul_quantize: need m >= 0 and f a positive multiple of 32 "
+                                           "(m=%lld f=%lld)", (long long)m, (long long)f);
+    if (m >= (1ll << 31) || f >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "silu_mul_quantize: dimension >= 2^31");
+    if (ldgu < f) return fail(NVFP4_ERR_INVALID_ARG, "silu_mul_quantize: ldgu %lld < f %lld", (long long)ldgu,
+                              (long long)f);
+    if (h_out != nullptr && ldh < f)
+        return fail(NVFP4_ERR_INVALID_ARG, "silu_mul_quantize: ldh %lld < f %lld", (long long)ldh, (long long)f);
+    if (m > 0 && (g == nullptr || u == nullptr || h_q == nullptr || h_sf == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "silu_mul_quantize: NULL input or output pointer");
+    if (!aligned16(g) || !aligned16(u) || (ldgu * 2) % 16 != 0 || !aligned16(h_q) || !aligned16(h_sf) ||
+        !aligned16(h_out) || (h_out != nullptr && (ldh * 2) % 16 != 0))
+        return fail(NVFP4_ERR_ALIGNMENT, "silu_mul_quantize: rows and outputs must be 16-byte aligned");
+    const bool dynamic = h_scale_dev == nullptr;
+    if (dynamic) {
+        if (h_scale_out_dev == nullptr)
+            return fail(NVFP4_ERR_INVALID_ARG, "silu_mul_quantize: dynamic mode needs h_scale_out_dev");
+        if (workspace == nullptr || ws_bytes < nvfp4_quant_workspace_size())
+            return fail(NVFP4_ERR_WORKSPACE, "silu_mul_quantize: dynamic mode needs %zu bytes of workspace",
+                        nvfp4_quant_workspace_size());
+        if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "silu_mul_quantize: workspace not 16-byte aligned");
+    }
+    if (m == 0) return ok();
+    DeviceState* dev = nullptr;
+    nvfp4_status st = device_state(&dev);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    QuantParams p = {};
+    p.x = g;
+    p.rows = m;
+    p.k = f;
+    p.ldx = ldgu;
+    p.q = h_q;
+    p.sf = h_sf;
+    p.sf_rows_end = pad_to(m, 128);
+    p.scale_mode = dynamic ? kScaleFromAmax : kScaleDevice;
+    p.scale_ptr = dynamic ? static_cast<const float*>(workspace) : h_scale_dev;
+    p.scale_out = h_scale_out_dev;
+    SiluParams sp;
+    sp.g = static_cast<const __nv_bfloat16*>(g);
+    sp.u = static_cast<const __nv_bfloat16*>(u);
+    sp.ldgu = ldgu;
+    sp.h = static_cast<__nv_bfloat16*>(h_out);
+    sp.ldh = ldh;
+    if (dynamic) {
+        // pass 1: amax of h (h itself is stored here when asked for)
+        NVFP4_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(unsigned int), s));
+        if ((st = launch_quant(p, s, kAmaxSiluMul, &sp, static_cast<unsigned int*>(workspace))) != NVFP4_OK)
+            return st;
+        sp.h = nullptr;
+    }
+    if ((st = launch_quant(p, s, kQuantSiluMul, &sp)) != NVFP4_OK) return st;
     return ok();
 }
 

@@ -210,11 +210,37 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& a, float* v)
     }
 }
 
+// Quantise the two blocks a thread holds and store their codes and, from the
+// even lane of each lane pair, the 32-bit scale word of four blocks.  Must be
+// reached by every lane of the warp (the scale bytes are exchanged by shuffle).
+__device__ __forceinline__ void quantize_pair_store(const QuantParams& p, const QuantLaunch& l, bool mapped,
+                                                    uint32_t pr, int64_t r, int64_t kb0, bool live0, bool live1,
+                                                    float s_g, const float (&v0)[16], const float (&v1)[16])
+{
+    uint32_t sb0, sb1;
+    uint2 q0, q1;
+    quantize_block16(v0, s_g, live0, sb0, q0);
+    quantize_block16(v1, s_g, live1, sb1, q1);
+    const int64_t grow = p.row_offset + r;
+    uint8_t* qdst = p.q + grow * (p.k >> 1) + kb0 * 8;
+    if (live1)
+        *reinterpret_cast<uint4*>(qdst) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    else if (live0)
+        *reinterpret_cast<uint2*>(qdst) = q0;
+
+    // Four consecutive blocks form one 32-bit word of an atom row.
+    const uint32_t half = sb0 | (sb1 << 8);
+    const uint32_t other = __shfl_down_sync(0xffffffffu, half, 1);
+    if (mapped && (pr & 1u) == 0u) {
+        const uint32_t word = half | (other << 16);
+        *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb0, l.pairs >> 1)) = word;
+    }
+}
+
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p,
                                                                const QuantLaunch l)
 {
     const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
-    const uint32_t lane = threadIdx.x & 31u;
     const bool mapped = t < l.total;
     const uint32_t rl = mapped ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
     const uint32_t pr = mapped ? t - rl * l.pairs : 0u;
@@ -253,24 +279,130 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_co
         unpack_bf16x8(u[3], v1 + 8);
     }
 
-    uint32_t sb0, sb1;
-    uint2 q0, q1;
-    quantize_block16(v0, s_g, live0, sb0, q0);
-    quantize_block16(v1, s_g, live1, sb1, q1);
-    const int64_t grow = p.row_offset + r;
-    uint8_t* qdst = p.q + grow * (p.k >> 1) + kb0 * 8;
-    if (live1)
-        *reinterpret_cast<uint4*>(qdst) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    else if (live0)
-        *reinterpret_cast<uint2*>(qdst) = q0;
+    quantize_pair_store(p, l, mapped, pr, r, kb0, live0, live1, s_g, v0, v1);
+}
 
-    // Four consecutive blocks form one 32-bit word of an atom row.
-    const uint32_t half = sb0 | (sb1 << 8);
-    const uint32_t other = __shfl_down_sync(0xffffffffu, half, 1);
-    if (mapped && (pr & 1u) == 0u) {
-        const uint32_t word = half | (other << 16);
-        *reinterpret_cast<uint32_t*>(p.sf + sf_tiled_offset(grow, kb0, l.pairs >> 1)) = word;
+// ---------------------------------------------------------------------------
+// MLP glue: h = bf16(silu(g) * u) with silu(x) = x / (1 + e^-x), each step in
+// FP32 with round-to-nearest (e^-x from CUDA's expf), from the BF16 gate and up
+// halves of a fused gate/up GEMM output; h is then quantised like an
+// activation with its own tensor scale.  Same thread mapping as
+// quantize_kernel: one thread per two 16-element blocks of one row.
+// ---------------------------------------------------------------------------
+struct SiluParams {
+    const __nv_bfloat16* g;   // rows x f, row stride ldgu
+    const __nv_bfloat16* u;   // rows x f, row stride ldgu
+    int64_t ldgu;
+    __nv_bfloat16* h;         // optional rows x f output, row stride ldh (nullptr: not written)
+    int64_t ldh;
+};
+
+// h as the float value of its BF16 rounding.
+__device__ __forceinline__ float silu_mul_bf16(float g, float u)
+{
+    const float e = expf(-g);
+    const float s = __fdiv_rn(g, __fadd_rn(1.0f, e));
+    return __bfloat162float(__float2bfloat16_rn(__fmul_rn(s, u)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16_pair(float lo, float hi)
+{
+    return (__float_as_uint(lo) >> 16) | (__float_as_uint(hi) & 0xFFFF0000u);  // both already BF16 values
+}
+
+// Load the thread's 32 gate and 32 up values, form h for both blocks and, if
+// requested, store h.
+__device__ __forceinline__ void silu_mul_pair(const SiluParams& sp, int64_t r, int64_t kb0, bool live0, bool live1,
+                                              float (&v0)[16], float (&v1)[16])
+{
+    const uint4* gs = reinterpret_cast<const uint4*>(sp.g + r * sp.ldgu + kb0 * 16);
+    const uint4* us = reinterpret_cast<const uint4*>(sp.u + r * sp.ldgu + kb0 * 16);
+    uint4 gw[4], uw[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const bool live = (j < 2) ? live0 : live1;
+        gw[j] = live ? __ldcs(gs + j) : make_uint4(0, 0, 0, 0);
+        uw[j] = live ? __ldcs(us + j) : make_uint4(0, 0, 0, 0);
     }
+    float gf[32], uf[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        unpack_bf16x8(gw[j], gf + 8 * j);
+        unpack_bf16x8(uw[j], uf + 8 * j);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        v0[e] = silu_mul_bf16(gf[e], uf[e]);
+        v1[e] = silu_mul_bf16(gf[16 + e], uf[16 + e]);
+    }
+    if (sp.h != nullptr) {
+        uint4* hd = reinterpret_cast<uint4*>(sp.h + r * sp.ldh + kb0 * 16);
+        if (live0) {
+            hd[0] = make_uint4(pack_bf16_pair(v0[0], v0[1]), pack_bf16_pair(v0[2], v0[3]),
+                               pack_bf16_pair(v0[4], v0[5]), pack_bf16_pair(v0[6], v0[7]));
+            hd[1] = make_uint4(pack_bf16_pair(v0[8], v0[9]), pack_bf16_pair(v0[10], v0[11]),
+                               pack_bf16_pair(v0[12], v0[13]), pack_bf16_pair(v0[14], v0[15]));
+        }
+        if (live1) {
+            hd[2] = make_uint4(pack_bf16_pair(v1[0], v1[1]), pack_bf16_pair(v1[2], v1[3]),
+                               pack_bf16_pair(v1[4], v1[5]), pack_bf16_pair(v1[6], v1[7]));
+            hd[3] = make_uint4(pack_bf16_pair(v1[8], v1[9]), pack_bf16_pair(v1[10], v1[11]),
+                               pack_bf16_pair(v1[12], v1[13]), pack_bf16_pair(v1[14], v1[15]));
+        }
+    }
+}
+
+// Pass 1 of the dynamic-scale glue: amax of h (optionally storing h).
+__global__ void __launch_bounds__(kQuantThreads) silu_mul_amax_kernel(const __grid_constant__ QuantParams p,
+                                                                    const __grid_constant__ SiluParams sp,
+                                                                    const QuantLaunch l, unsigned int* amax)
+{
+    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
+    const bool mapped = t < l.total;
+    const uint32_t rl = mapped ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
+    const uint32_t pr = mapped ? t - rl * l.pairs : 0u;
+    const int64_t r = l.row_begin + rl;
+    const int64_t kb0 = (int64_t)pr * 2;
+    const bool row_live = mapped && r < p.rows;
+    const bool live0 = row_live && kb0 < (p.k >> 4);
+    const bool live1 = row_live && kb0 + 1 < (p.k >> 4);
+    float v0[16], v1[16];
+    silu_mul_pair(sp, r, kb0, live0, live1, v0, v1);
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) m = fmaxf(m, fmaxf(fabsf(v0[e]), fabsf(v1[e])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float red[kQuantThreads / 32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = 0.0f;
+        for (int i = 0; i < kQuantThreads / 32; ++i) b = fmaxf(b, red[i]);
+        if (b > 0.0f) atomicMax(amax, __float_as_uint(b));
+    }
+}
+
+// h = bf16(silu(g) * u) quantised to NVFP4 (optionally storing h).
+__global__ void __launch_bounds__(kQuantThreads) silu_mul_quantize_kernel(const __grid_constant__ QuantParams p,
+                                                                        const __grid_constant__ SiluParams sp,
+                                                                        const QuantLaunch l)
+{
+    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
+    const bool mapped = t < l.total;
+    const uint32_t rl = mapped ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
+    const uint32_t pr = mapped ? t - rl * l.pairs : 0u;
+    const int64_t r = l.row_begin + rl;
+    const int64_t kb0 = (int64_t)pr * 2;
+    const bool row_live = mapped && r < p.rows;
+    const bool live0 = row_live && kb0 < (p.k >> 4);
+    const bool live1 = row_live && kb0 + 1 < (p.k >> 4);
+
+    const float s_g = load_scale(p);
+    if (p.scale_out != nullptr && t == 0 && l.row_begin == 0) *p.scale_out = s_g;
+    float v0[16], v1[16];
+    silu_mul_pair(sp, r, kb0, live0, live1, v0, v1);
+    quantize_pair_store(p, l, mapped, pr, r, kb0, live0, live1, s_g, v0, v1);
 }
 
 }  // namespace nvfp4

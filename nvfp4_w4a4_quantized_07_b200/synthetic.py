@@ -119,6 +119,16 @@ def mlp_down_weight(k: int = MLP_INTERMEDIATE, n: int = HIDDEN) -> torch.Tensor:
     return weights(n, k, 0.02, seed=3)
 
 
+def mlp_glue_inputs(m: int, f: int, seed: int = 5, gate_std: float = 2.0) -> torch.Tensor:
+    """A fused ``[gate | up]`` BF16 tensor of shape ``m x 2f`` (gate N(0, gate_std^2),
+    up N(0, 1)), the shape of a fused gate/up GEMM output."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    gate = torch.randn(m, f, generator=g, dtype=torch.float32) * gate_std
+    up = torch.randn(m, f, generator=g, dtype=torch.float32)
+    return torch.cat([gate, up], dim=1).to(torch.bfloat16).contiguous()
+
+
 DECODE_SHAPES = {
     # name: (list of module widths, K, list of stds)
     "5120x5120": ([5120], HIDDEN, [0.02]),

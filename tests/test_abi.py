@@ -180,3 +180,17 @@ def test_decode_noalloc_limits_without_a_device(lib):
     assert nv.NVFP4_NOALLOC_MAX_M == 16
     # the built-in scratch is exactly the decode workspace for 16 tokens
     assert lib.nvfp4_gemm_workspace_size(16, 64, 64, nv.NVFP4_GEMM_FORCE_DECODE) == 2048 + 256 * 16 * 256 * 4
+
+
+def test_silu_mul_quantize_argument_errors(lib):
+    f = lib.nvfp4_silu_mul_quantize
+    ws = ctypes.c_void_p(0x20000)
+    assert f(FAKE, FAKE, 8, 48, 96, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 1     # f % 32
+    assert f(FAKE, FAKE, 8, 64, 32, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 1     # ldgu < f
+    assert f(None, FAKE, 8, 64, 128, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 1    # null g
+    assert f(FAKE, FAKE, 8, 64, 128, FAKE, None, FAKE, FAKE, FAKE, 32, None, 0, None) == 1   # ldh < f
+    assert f(FAKE, MISALIGNED, 8, 64, 128, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 3
+    assert f(FAKE, FAKE, 8, 64, 68, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 3     # row pitch
+    assert f(FAKE, FAKE, 8, 64, 128, None, None, FAKE, FAKE, None, 0, ws, 256, None) == 1    # dynamic: no scale out
+    assert f(FAKE, FAKE, 8, 64, 128, None, FAKE, FAKE, FAKE, None, 0, None, 0, None) == 6    # dynamic: no workspace
+    assert f(FAKE, FAKE, 0, 64, 128, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 0    # empty
