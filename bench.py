@@ -69,10 +69,10 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the GEMM kernel's device source (the counters of a profile hold
-    only for the source they were taken on)."""
+    """Hash of the large-M GEMM kernel's device source (the counters of a
+    profile hold only for the source they were taken on)."""
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "ptx.cuh"):
+    for f in ("gemm_common.cuh", "gemm_large.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_07_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

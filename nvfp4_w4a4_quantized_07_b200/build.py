@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4.so")
 SOURCES = [os.path.join(CSRC, "nvfp4_lib.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quant.cuh", "gemm.cuh")] + \
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quant.cuh", "gemm_common.cuh", "gemm_large.cuh", "gemm_decode.cuh")] + \
     [os.path.join(ROOT, "include", "nvfp4.h")]
 
 

@@ -1,6 +1,6 @@
 // libnvfp4: the C ABI declared in include/nvfp4.h.  Argument validation, TMA
 // descriptor creation and kernel launches; all arithmetic runs in the kernels
-// of quant.cuh and gemm.cuh.  Single translation unit.
+// of quant.cuh, gemm_large.cuh and gemm_decode.cuh.  Single translation unit.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -15,7 +15,8 @@
 #include <random>
 
 #include "../../include/nvfp4.h"
-#include "gemm.cuh"
+#include "gemm_decode.cuh"
+#include "gemm_large.cuh"
 #include "quant.cuh"
 
 using namespace nvfp4;
