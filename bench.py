@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-mlp", action="store_true", help="skip the prefill and long-prefill MLP measurements")
     ap.add_argument("--profile-gemm", action="store_true",
                     help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
+    ap.add_argument("--probe-peaks", action="store_true",
+                    help="measure the dense FP4 tensor-core rate and the HBM read rate with the probe kernels")
     ap.add_argument("--decode-case", default=None,
                     help="time one decode GEMM only, e.g. m16_5120x5120 (for ncu captures)")
     return ap.parse_args()
@@ -472,7 +474,8 @@ def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
     c1 = torch.empty((p.m, 2 * f), dtype=torch.bfloat16, device=device)
     c2 = torch.empty((p.m, p.k), dtype=torch.bfloat16, device=device)
     ws = nv.quant_workspace(device)
-    hq = nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws)[0]
+    h = torch.empty((p.m, f), dtype=torch.bfloat16, device=device)
+    hq = nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws, h_out=h)[0]
 
     def stage(i):
         if i == 0:
@@ -480,7 +483,7 @@ def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
         elif i == 1:
             nv.gemm(aq, fw1, out=c1)
         elif i == 2:
-            nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws, out=hq)
+            nv.silu_mul_quantize(c1[:, :f], c1[:, f:], workspace=ws, out=hq, h_out=h)
         else:
             nv.gemm(hq, fw2, out=c2)
 
@@ -491,7 +494,7 @@ def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
     ms = _timed(mlp_step, flush, stream, device, reps=3, warm=1)
     flops = 2.0 * p.m * (2 * f) * p.k + 2.0 * p.m * p.k * f
     glue_ms = _timed(lambda: stage(2), flush, stream, device, reps=3, warm=1)
-    glue_bytes = p.m * f * (2 * 2 * 2 + 0.5 + 1 / 16)      # g, u read twice (dynamic), codes + scales written
+    glue_bytes = p.m * f * (2 * 2 + 2 + 2 + 0.5 + 1 / 16)  # g, u read; h written and read back; codes + scales
     res["mlp_32768x5120_17408"] = {
         "value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
         "gemm_gate_up_ms": _timed(lambda: stage(1), flush, stream, device, reps=3, warm=1),
@@ -499,6 +502,72 @@ def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
         "glue_ms": glue_ms, "glue_GB/s": glue_bytes / (glue_ms * 1e-3) / 1e9,
         "glue_frac_hbm": glue_bytes / (glue_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     return res
+
+
+def run_probe_peaks(args):
+    """Roofline denominators measured by libnvfp4_probes: the dense
+    block-scaled FP4 MMA rate (operands resident in shared memory, one CTA per
+    SM) and the read-only HBM streaming rate (4 GiB buffer)."""
+    import ctypes
+
+    import torch
+
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+
+    lib = ctypes.CDLL(nvbuild.build_probes())
+    P = ctypes.c_void_p
+    lib.nvfp4_probe_mma_peak.argtypes = [ctypes.c_int, ctypes.c_int, P, P]
+    lib.nvfp4_probe_mma_peak_pair.argtypes = [ctypes.c_int, ctypes.c_int, P, P]
+    lib.nvfp4_probe_hbm_read.argtypes = [P, ctypes.c_longlong, P, ctypes.c_int, P]
+    lib.nvfp4_probe_status.argtypes = [P]
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(device)
+    sp = P(stream.cuda_stream)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    cycles = torch.zeros(1, dtype=torch.int64, device=device)
+
+    def timed(launch, reps):
+        times = []
+        for it in range(reps + 2):
+            torch.cuda._sleep(500_000)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            rc = launch()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            if rc != 0:
+                raise RuntimeError(f"probe launch failed: cudaError {rc}")
+            if it >= 2:
+                times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    iters = 16384
+    with ClockSampler(0) as clk_mma:
+        mma_ms = timed(lambda: lib.nvfp4_probe_mma_peak(iters, sms, P(cycles.data_ptr()), sp), max(args.steps, 5))
+    mma_flops = 2.0 * 128 * 256 * 64 * 4 * iters * sms
+    cyc = int(cycles.item())
+    pair_ms = timed(lambda: lib.nvfp4_probe_mma_peak_pair(iters, sms - sms % 2, P(cycles.data_ptr()), sp),
+                    max(args.steps, 5))
+    pair_flops = 2.0 * 256 * 256 * 64 * 4 * iters * (sms // 2)
+    pair_cyc = int(cycles.item())
+    buf = torch.randint(0, 256, (4 << 30,), dtype=torch.uint8, device=device)
+    sink = torch.zeros(1, dtype=torch.int32, device=device)
+    with ClockSampler(0) as clk_hbm:
+        hbm_ms = timed(lambda: lib.nvfp4_probe_hbm_read(P(buf.data_ptr()), buf.numel(), P(sink.data_ptr()), sms * 8,
+                                                        sp), max(args.steps, 5))
+    status = ctypes.c_uint(0)
+    lib.nvfp4_probe_status(ctypes.byref(status))
+    print(json.dumps({
+        "probe": "peaks", "sms": sms, "status": int(status.value),
+        "fp4_mma": {"tflops": mma_flops / (mma_ms * 1e-3) / 1e12, "ms": mma_ms,
+                    "cycles_per_mma_cta0": cyc / (4 * iters), "mma": "M128 N256 K64 kind::mxf4nvf4, cta_group::1",
+                    "clocks": clk_mma.summary()},
+        "fp4_mma_pair": {"tflops": pair_flops / (pair_ms * 1e-3) / 1e12, "ms": pair_ms,
+                         "cycles_per_mma_pair0": pair_cyc / (4 * iters),
+                         "mma": "M256 N256 K64 kind::mxf4nvf4, cta_group::2"},
+        "hbm_read": {"GB/s": buf.numel() / (hbm_ms * 1e-3) / 1e9, "ms": hbm_ms, "bytes": buf.numel(),
+                     "clocks": clk_hbm.summary()}}), flush=True)
+    return 0
 
 
 def run_decode_case(args):
@@ -544,6 +613,8 @@ def main():
         return run_reference(args)
     if args.decode_case:
         return run_decode_case(args)
+    if args.probe_peaks:
+        return run_probe_peaks(args)
     return run_ours(args)
 
 

@@ -213,7 +213,9 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
  *   workspace         device, >= nvfp4_quant_workspace_size() bytes, needed
  *                     only in dynamic mode.
  * Shapes: m >= 0, f a positive multiple of 32, both < 2^31.
- * Dynamic mode reads g and u twice (amax pass, then the quantising pass).
+ * Dynamic mode runs an amax pass first.  With h_out it stores h there and
+ * quantises the stored h (silu evaluated once per element); without h_out it
+ * reads g and u again and recomputes h.  The bytes are the same either way.
  * ---------------------------------------------------------------------- */
 NVFP4_API nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int64_t m, int64_t f, int64_t ldgu,
                                      const float* h_scale_dev, float* h_scale_out_dev, uint8_t* h_q, uint8_t* h_sf,

@@ -174,12 +174,13 @@ def quantize_act(a, act_scale=None, workspace=None, out: QuantizedActivation | N
 
 
 def silu_mul_quantize(g, u, h_scale=None, return_h: bool = False, workspace=None,
-                      out: QuantizedActivation | None = None):
+                      out: QuantizedActivation | None = None, h_out=None):
     """MLP glue (``nvfp4_silu_mul_quantize``): h = bf16(silu(g) * u) quantised
     to NVFP4.  ``g`` and ``u`` are BF16 m x f CUDA tensors with unit column
     stride and the same row stride (e.g. the two halves of a fused gate/up
     GEMM output).  ``h_scale`` is a static 1-element FP32 device scale or
-    ``None`` (dynamic).  Returns ``(QuantizedActivation, h or None)``."""
+    ``None`` (dynamic).  ``h_out`` (a contiguous m x f BF16 tensor) or
+    ``return_h`` also stores h.  Returns ``(QuantizedActivation, h or None)``."""
     import torch
     _require_cuda(g, u, h_scale)
     if g.dtype != torch.bfloat16 or u.dtype != torch.bfloat16:
@@ -193,7 +194,11 @@ def silu_mul_quantize(g, u, h_scale=None, return_h: bool = False, workspace=None
             q=torch.empty((m, f // 2), dtype=torch.uint8, device=g.device),
             sf=torch.empty(max(L.nvfp4_sf_bytes(m, f), 1), dtype=torch.uint8, device=g.device),
             scale=torch.empty(1, dtype=torch.float32, device=g.device), m=m, k=f)
-    h = torch.empty((m, f), dtype=torch.bfloat16, device=g.device) if return_h else None
+    h = h_out
+    if h is None and return_h:
+        h = torch.empty((m, f), dtype=torch.bfloat16, device=g.device)
+    if h is not None and (h.shape != (m, f) or h.dtype != torch.bfloat16 or not h.is_contiguous()):
+        raise ValueError("h_out must be a contiguous m x f bfloat16 tensor")
     if h_scale is None and workspace is None:
         workspace = quant_workspace(g.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

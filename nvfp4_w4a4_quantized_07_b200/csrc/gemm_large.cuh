@@ -24,16 +24,45 @@ namespace nvfp4 {
 // TMEM (512 columns): two 256-column accumulators overlapping by 96 columns,
 // ACC0 = [0, 256) and ACC1 = [160, 416), and two 48-column scale slots at
 // [416, 512).  Consecutive tiles alternate accumulators; the epilogue drains
-// the shared 96 columns first and releases them, so the next tile's MMAs start
-// while the rest of the previous tile is still being drained.
+// the shared columns first and releases them, so the next tile's MMAs start
+// while the rest of the previous tile is still being drained.  (A larger
+// overlap with more scale slots, [64, 320) and four slots, measured slower:
+// the longer drain before the next tile's first MMA costs more than the
+// deeper scale staging gains.)
 // ===========================================================================
+// Overlap plan for accumulators ACC0 = [0, 256) and ACC1 = [A1, A1 + 256)
+// (A1 a multiple of 32): the 32-column chunks of each epilogue warp's
+// 128-column half that the other accumulator also uses.  They are drained
+// first, starting at chunk rot(b, h); after count(b, h) of them the warp
+// releases the overlap (count 0: the warp holds none).
+template <int A1>
+struct Overlap {
+    static constexpr int b0_from = A1 / 32;          // ACC0 chunks >= b0_from are shared
+    static constexpr int b1_to = (256 - A1) / 32;    // ACC1 chunks < b1_to are shared
+    __host__ __device__ static constexpr int clamp4(int x) { return x < 0 ? 0 : (x > 4 ? 4 : x); }
+    __host__ __device__ static constexpr int count(int b, int h)
+    {
+        return b == 0 ? clamp4(4 * h + 4 - (b0_from > 4 * h ? b0_from : 4 * h))
+                      : clamp4((b1_to < 4 * h + 4 ? b1_to : 4 * h + 4) - 4 * h);
+    }
+    __host__ __device__ static constexpr int rot(int b, int h)
+    {
+        return (b == 0 && count(0, h) > 0 && b0_from > 4 * h) ? (b0_from - 4 * h) & 3 : 0;
+    }
+    // warps that release the overlap per tile (the same for both accumulators)
+    __host__ __device__ static constexpr int warps() { return 4 * ((count(0, 0) > 0) + (count(0, 1) > 0)); }
+    static_assert(A1 % 32 == 0 && A1 > 0 && A1 < 256, "overlap");
+    static_assert(4 * ((count(0, 0) > 0) + (count(0, 1) > 0)) == 4 * ((count(1, 0) > 0) + (count(1, 1) > 0)),
+                  "both accumulators release through the same number of warps");
+};
+
 // Drain one warp's 32 x 128 slice of an accumulator into scaled BF16 pairs,
 // 32 columns at a time starting with chunk ROT (compile-time so the results
-// stay in registers).  After the third chunk the warp optionally arrives on
-// `after3` (the columns shared with the other accumulator are then free).
-template <int ROT>
+// stay in registers).  After AFTER chunks (0: never) the warp calls
+// `release()` (the columns shared with the other accumulator are then free).
+template <int ROT, int AFTER, typename Release>
 __device__ __forceinline__ void drain_bf16(uint32_t taddr, int ncol0, float s_ga, const GemmParams& p,
-                                           uint64_t* after3, int lane, uint32_t (&packed)[4][16])
+                                           Release release, int lane, uint32_t (&packed)[4][16])
 {
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -41,10 +70,10 @@ __device__ __forceinline__ void drain_bf16(uint32_t taddr, int ncol0, float s_ga
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + j * 32, v);
         tmem_ld_wait();
-        if (jj == 2 && after3 != nullptr) {
+        if (jj + 1 == AFTER) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(after3);
+            if (lane == 0) release();
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -55,6 +84,26 @@ __device__ __forceinline__ void drain_bf16(uint32_t taddr, int ncol0, float s_ga
                 packed[j][h * 8 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h * 16 + 2 * e]), alpha),
                                                    __fmul_rn(__uint_as_float(v[h * 16 + 2 * e + 1]), alpha));
         }
+    }
+}
+
+// Dispatch drain_bf16 on the (accumulator, half) overlap plan.
+template <int A1, typename Release>
+__device__ __forceinline__ void drain_bf16_plan(int b, int half, uint32_t taddr, int ncol0, float s_ga,
+                                                const GemmParams& p, Release release, int lane,
+                                                uint32_t (&packed)[4][16])
+{
+    using OV = Overlap<A1>;
+    if (b == 0) {
+        if (half == 0)
+            drain_bf16<OV::rot(0, 0), OV::count(0, 0)>(taddr, ncol0, s_ga, p, release, lane, packed);
+        else
+            drain_bf16<OV::rot(0, 1), OV::count(0, 1)>(taddr, ncol0, s_ga, p, release, lane, packed);
+    } else {
+        if (half == 0)
+            drain_bf16<OV::rot(1, 0), OV::count(1, 0)>(taddr, ncol0, s_ga, p, release, lane, packed);
+        else
+            drain_bf16<OV::rot(1, 1), OV::count(1, 1)>(taddr, ncol0, s_ga, p, release, lane, packed);
     }
 }
 
@@ -73,8 +122,9 @@ constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_C = OFF_SFB + STAGES * SFB_STAGE;
 constexpr int C_WARP = 1024;                       // per epilogue warp: one 16 x 32 BF16 chunk
 constexpr int OFF_BAR = OFF_C + 8 * C_WARP;
-// full[S], empty[S], sf_ready[2], sf_free[2], acc_full[2], acc_empty[2], ovl_free, drain
-constexpr int NUM_BARS = 2 * STAGES + 2 + 2 + 2 + 2 + 1 + 1;
+constexpr int SF_SLOTS = 2;
+// full[S], empty[S], sf_ready[SLOTS], acc_full[2], acc_empty[2], ovl_free, drain
+constexpr int NUM_BARS = 2 * STAGES + SF_SLOTS + 2 + 2 + 1 + 1;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;  // + alignment slack
 constexpr int THREADS = 512;
@@ -82,7 +132,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC1_COL = 160;                         // ACC0 at 0; overlap [160, 256)
 constexpr int SF_COL = 416;                           // two scale slots of 48 columns
 constexpr int SF_SLOT = 48;                           // 16 (A: 4 k-steps x 4) + 32 (B: 4 x 8)
-static_assert(ACC1_COL + BN <= SF_COL && SF_COL + 2 * SF_SLOT <= TMEM_COLS, "TMEM budget");
+static_assert(ACC1_COL + BN <= SF_COL && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace large
 
@@ -96,8 +146,7 @@ __global__ void __launch_bounds__(large::THREADS, 1)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* empty = full + STAGES;
     uint64_t* sf_ready = empty + STAGES;
-    uint64_t* sf_free = sf_ready + 2;
-    uint64_t* acc_full = sf_free + 2;
+    uint64_t* acc_full = sf_ready + SF_SLOTS;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* ovl_free = acc_empty + 2;
     uint64_t* drain = ovl_free + 1;
@@ -115,13 +164,14 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < SF_SLOTS; ++i) {
             mbar_init(&sf_ready[i], 4);
-            mbar_init(&sf_free[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 8);
         }
-        mbar_init(ovl_free, 4);
+        mbar_init(ovl_free, Overlap<ACC1_COL>::warps());
         mbar_init(drain, 1);
         fence_mbarrier_init();
     }
@@ -181,8 +231,10 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_nvf4(BM, BN);
+            const uint64_t adesc0 = desc_kmajor_sw128(smem + OFF_A);
+            const uint64_t bdesc0 = desc_kmajor_sw128(smem + OFF_B);
             int stage = 0, slot = 0;
-            uint32_t phase = 0, slot_phase = 0;
+            uint32_t slot_phase = 0;
             bool ok = true;
             int i = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++i) {
@@ -202,22 +254,27 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
                     const uint32_t sf_col = tmem_base + SF_COL + slot * SF_SLOT;
-                    const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
-                    const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
-                    for (int ks = 0; ks < nks; ++ks) {
-                        // 64 FP4 values = 32 bytes along K: +2 in the descriptor's 16-byte units.
-                        mma_nvf4(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0, sf_col + 4 * ks,
-                                 sf_col + 16 + 8 * ks);
+                    // stage buffers are 1 KB aligned: advance the descriptors' address fields
+                    const uint64_t adesc = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
+                    const uint64_t bdesc = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
+                    // 64 FP4 values = 32 bytes along K: +2 in the descriptor's 16-byte units.
+                    if (kt + 1 < p.k_tiles || p.katoms % KSTEPS == 0) {
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+                            mma_nvf4(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0, sf_col + 4 * ks,
+                                     sf_col + 16 + 8 * ks);
+                    } else {
+                        const int nks = p.katoms - kt * KSTEPS;
+                        for (int ks = 0; ks < nks; ++ks)
+                            mma_nvf4(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0, sf_col + 4 * ks,
+                                     sf_col + 16 + 8 * ks);
                     }
+                    // one commit frees the stage for the producer and, for the
+                    // scale warps, the scale slot these MMAs read
                     mma_commit(&empty[stage]);
-                    mma_commit(&sf_free[slot]);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                    if (++slot == 2) {
+                    if (++stage == STAGES) stage = 0;
+                    if (++slot == SF_SLOTS) {
                         slot = 0;
                         slot_phase ^= 1;
                     }
@@ -230,7 +287,6 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                 mma_commit(drain);
                 mbar_wait(drain, 0, kStatusTimeoutDrain, kWaitCycles / 8);
             }
-            (void)phase;
         }
         __syncwarp();
     } else if (warp >= 12) {
@@ -238,14 +294,20 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         // Quadrant q writes lanes 32q..32q+31; each lane l receives row l of every
         // atom (16 bytes = the scales of rows l, l+32, l+64, l+96), which is the
         // layout block-scaled MMAs read for both operands.
+        // The slot of stage k was last read by the MMAs of stage k - SF_SLOTS;
+        // their completion is the commit on that stage's empty barrier (which
+        // cannot run a phase ahead: stage k + SF_SLOTS needs this slot first).
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         int stage = 0, slot = 0;
-        uint32_t phase = 0, slot_phase = 0;
+        uint32_t phase = 0;
+        long long kglob = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            for (int kt = 0; kt < p.k_tiles; ++kt) {
+            for (int kt = 0; kt < p.k_tiles; ++kt, ++kglob) {
+                const long long kprev = kglob - SF_SLOTS;
                 if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull) ||
-                    !mbar_wait(&sf_free[slot], slot_phase ^ 1, kStatusTimeoutFull)) {
+                    (kprev >= 0 && !mbar_wait(&empty[kprev % STAGES], (uint32_t)((kprev / STAGES) & 1),
+                                              kStatusTimeoutFull))) {
                     ok = false;
                     break;
                 }
@@ -285,10 +347,7 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                     stage = 0;
                     phase ^= 1;
                 }
-                if (++slot == 2) {
-                    slot = 0;
-                    slot_phase ^= 1;
-                }
+                if (++slot == SF_SLOTS) slot = 0;
             }
         }
     } else if (warp >= 4) {
@@ -306,17 +365,14 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             const int row = mb * BM + quad * 32 + lane;
             const int ncol0 = nb * BN + half * 128;
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (b ? ACC1_COL : 0) + half * 128;
-            // The 96 columns shared with the other accumulator: ACC0's columns
-            // 160..255 (chunks 1-3 of half 1) or ACC1's columns 0..95 (chunks 0-2
-            // of half 0).  Their owners drain them first and release them.
-            const bool owns_overlap = half == (b == 0 ? 1 : 0);
-            const int first = (b == 0) ? 1 : 0;
+            // The columns shared with the other accumulator are drained first
+            // and released (Overlap<ACC1_COL>).
+            using OV = Overlap<ACC1_COL>;
+            const int ov_rot = OV::rot(b, half), ov_count = OV::count(b, half);
             if (!p.out_fp32) {
                 uint32_t packed[4][16];
-                if (owns_overlap && first == 1)
-                    drain_bf16<1>(taddr, ncol0, s_ga, p, ovl_free, lane, packed);
-                else
-                    drain_bf16<0>(taddr, ncol0, s_ga, p, owns_overlap ? ovl_free : nullptr, lane, packed);
+                drain_bf16_plan<ACC1_COL>(b, half, taddr, ncol0, s_ga, p, [&] { mbar_arrive(ovl_free); }, lane,
+                                          packed);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[b]);
@@ -349,11 +405,11 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                 }
             } else {
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = owns_overlap ? (first + jj) & 3 : jj;
+                    const int j = (ov_rot + jj) & 3;
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + j * 32, v);
                     tmem_ld_wait();
-                    if (owns_overlap && jj == 2) {
+                    if (jj + 1 == ov_count) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(ovl_free);
@@ -396,50 +452,60 @@ __global__ void __launch_bounds__(large::THREADS, 1)
 
 // ===========================================================================
 // Large-M kernel on CTA pairs (cta_group::2): a cluster of two CTAs on two SMs
-// computes a 256 x 256 tile with M = 256 MMAs.  Each CTA stages only its own
-// 128 rows of A and its own 128 rows of B (the pair's MMA reads both halves),
-// so each SM moves half the B bytes through shared memory per FLOP of the
-// single-CTA kernel; the even CTA issues the scale copies and MMAs for both.
-// Scale factors arrive by TMA too (3-D view: 512-byte atoms x K-atoms x
-// 128-row blocks), so out-of-range atoms are zero-filled by the copy engine.
+// computes a 256 x 256 tile with M = 256 MMAs issued by the even CTA.  Each CTA
+// stages its own 128 rows of A and its own 128 of the tile's 256 B rows, so per
+// FLOP an SM pulls 2/3 of the operand bytes of the single-CTA kernel through
+// L2 -> shared memory (the bound of that kernel).  The rest follows
+// gemm_large_kernel: scale staging with tcgen05.st in each CTA (its own A
+// scales and the full 256 rows of B scales, which its half of the MMA reads
+// from its own TMEM), overlapped accumulators, TMA-store epilogue on each
+// CTA's own 128 rows.  Each CTA's loads complete on its own barrier; the even
+// CTA learns that both halves of a stage are ready from the scale warps of
+// both CTAs (8 arrivals on its sf_ready), and its commits reach both CTAs.
 // ===========================================================================
 namespace pairk {
 constexpr int CTA_ROWS = 128, BN = 256, BK_BYTES = 128;
 constexpr int STAGES = 5;
 constexpr int KSTEPS = 4;
-constexpr int A_STAGE = CTA_ROWS * BK_BYTES;        // 16 KB: this CTA's half of the 256 A rows
-constexpr int B_STAGE = (BN / 2) * BK_BYTES;        // 16 KB: this CTA's half of the 256 B rows
+constexpr int A_STAGE = CTA_ROWS * BK_BYTES;        // 16 KB: this CTA's 128 of the 256 A rows
+constexpr int B_STAGE = (BN / 2) * BK_BYTES;        // 16 KB: this CTA's 128 of the 256 B rows
 constexpr int SFA_STAGE = 4 * 512;                  // 4 atoms of this CTA's 128 A rows
 constexpr int SFB_STAGE = 2 * 4 * 512;              // all 256 B rows: 2 row blocks x 4 atoms
-constexpr uint32_t STAGE_TX = A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE;
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int NUM_BARS = 2 * STAGES + 3;
+constexpr int OFF_C = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int C_WARP = 1024;
+constexpr int OFF_BAR = OFF_C + 8 * C_WARP;
+constexpr int SF_SLOTS = 2;
+// full[S], empty[S], sf_ready[SLOTS], acc_full[2], acc_empty[2], ovl_free, drain
+constexpr int NUM_BARS = 2 * STAGES + SF_SLOTS + 2 + 2 + 1 + 1;
 constexpr int OFF_TMEM_PTR = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_TMEM_PTR + 16 + 1024;
-constexpr int THREADS = 384;
+constexpr int THREADS = 512;
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_SF = 256;
-constexpr int TMEM_SF_STAGE = 48;
-static_assert(TMEM_SF + STAGES * TMEM_SF_STAGE <= TMEM_COLS, "TMEM budget");
+constexpr int ACC1_COL = 160;
+constexpr int SF_COL = 416;
+constexpr int SF_SLOT = 48;
+static_assert(ACC1_COL + BN <= SF_COL && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "TMEM budget");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace pairk
 
 __global__ void __launch_bounds__(pairk::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-                     const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfw,
-                     const __grid_constant__ GemmParams p)
+                     const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ GemmParams p)
 {
     using namespace pairk;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* empty = full + STAGES;
-    uint64_t* tmem_full = empty + STAGES;
-    uint64_t* tmem_empty = tmem_full + 1;
-    uint64_t* drain = tmem_empty + 1;
+    uint64_t* sf_ready = empty + STAGES;
+    uint64_t* acc_full = sf_ready + SF_SLOTS;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* ovl_free = acc_empty + 2;
+    uint64_t* drain = ovl_free + 1;
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + OFF_TMEM_PTR);
 
     const int warp = threadIdx.x >> 5;
@@ -452,14 +518,19 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensor_map(&tmap_a);
         prefetch_tensor_map(&tmap_w);
-        prefetch_tensor_map(&tmap_sfa);
-        prefetch_tensor_map(&tmap_sfw);
+        prefetch_tensor_map(&tmap_c);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 16);  // 8 epilogue warps in each CTA of the pair
+        for (int i = 0; i < SF_SLOTS; ++i) {
+            mbar_init(&sf_ready[i], 8);     // 4 scale warps in each CTA
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 16);   // 8 epilogue warps in each CTA
+        }
+        mbar_init(ovl_free, 2 * Overlap<ACC1_COL>::warps());
         mbar_init(drain, 1);
         fence_mbarrier_init();
     }
@@ -482,21 +553,32 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
                 const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
+                const int a_rb = 2 * mb + (int)rank;              // this CTA's 128-row block of A
+                const bool a_live = a_rb < p.a_rowblocks;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
                         ok = false;
                         break;
                     }
-                    // The stage's four copies of BOTH CTAs complete on the even CTA's barrier.
-                    const uint32_t bar0 = map_shared_rank(smem_u32(&full[stage]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_TX);
-                    tma_load_2d_pair(smem + OFF_A + stage * A_STAGE, &tmap_a, bar0, kt * BK_BYTES,
-                                     mb * 2 * CTA_ROWS + (int)rank * CTA_ROWS);
-                    tma_load_2d_pair(smem + OFF_B + stage * B_STAGE, &tmap_w, bar0, kt * BK_BYTES,
-                                     nb * BN + (int)rank * (BN / 2));
-                    tma_load_3d_pair(smem + OFF_SFA + stage * SFA_STAGE, &tmap_sfa, bar0, 0, kt * KSTEPS,
-                                     2 * mb + (int)rank);
-                    tma_load_3d_pair(smem + OFF_SFB + stage * SFB_STAGE, &tmap_sfw, bar0, 0, kt * KSTEPS, 2 * nb);
+                    const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
+                    const uint32_t sf_bytes = (uint32_t)nks * 512u;
+                    const bool w_rb1 = 2 * nb + 1 < p.w_rowblocks;
+                    const uint32_t bytes =
+                        A_STAGE + B_STAGE + sf_bytes * ((a_live ? 1u : 0u) + 1u + (w_rb1 ? 1u : 0u));
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES,
+                                a_rb * CTA_ROWS);
+                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES,
+                                nb * BN + (int)rank * (BN / 2));
+                    if (a_live)
+                        bulk_load(smem + OFF_SFA + stage * SFA_STAGE,
+                                  p.a_sf + ((int64_t)a_rb * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
+                    bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
+                              p.w_sf + ((int64_t)(2 * nb) * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
+                    if (w_rb1)
+                        bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
+                                  p.w_sf + ((int64_t)(2 * nb + 1) * p.katoms + kt * KSTEPS) * 512, sf_bytes,
+                                  &full[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -514,43 +596,51 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer (even CTA)
         if (lane == 0 && rank == 0) {
             const uint32_t idesc = idesc_nvf4(2 * CTA_ROWS, BN);
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            const uint64_t adesc0 = desc_kmajor_sw128(smem + OFF_A);
+            const uint64_t bdesc0 = desc_kmajor_sw128(smem + OFF_B);
+            int stage = 0, slot = 0;
+            uint32_t slot_phase = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-                if (!mbar_wait(tmem_empty, acc_phase ^ 1, kStatusTimeoutAccum)) {
+            int i = 0;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++i) {
+                const int b = i & 1;
+                if (!mbar_wait(&acc_empty[b], ((i >> 1) & 1) ^ 1, kStatusTimeoutAccum) ||
+                    (i > 0 && !mbar_wait(ovl_free, (i - 1) & 1, kStatusTimeoutAccum))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t acc = tmem_base + (b ? ACC1_COL : 0);
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull)) {
+                    // both CTAs' stage has landed and its scales are in both TMEMs
+                    if (!mbar_wait(&sf_ready[slot], slot_phase, kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
-                    const uint32_t sf_col = tmem_base + TMEM_SF + stage * TMEM_SF_STAGE;
-                    const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE;
-                    const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE;
-                    for (int ks = 0; ks < nks; ++ks) {
-                        tmem_cp_32x128b_x4_pair(sf_col + 4 * ks, desc_sf_atom(sfa + ks * 512));
-                        tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * ks, desc_sf_atom(sfb + ks * 512));
-                        tmem_cp_32x128b_x4_pair(sf_col + 16 + 8 * ks + 4, desc_sf_atom(sfb + 2048 + ks * 512));
+                    const uint32_t sf_col = tmem_base + SF_COL + slot * SF_SLOT;
+                    const uint64_t adesc = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
+                    const uint64_t bdesc = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
+                    if (kt + 1 < p.k_tiles || p.katoms % KSTEPS == 0) {
+#pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks)
+                            mma_nvf4_pair(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0,
+                                          sf_col + 4 * ks, sf_col + 16 + 8 * ks);
+                    } else {
+                        const int nks = p.katoms - kt * KSTEPS;
+                        for (int ks = 0; ks < nks; ++ks)
+                            mma_nvf4_pair(acc, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0,
+                                          sf_col + 4 * ks, sf_col + 16 + 8 * ks);
                     }
-                    const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
-                    const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
-                    for (int ks = 0; ks < nks; ++ks)
-                        mma_nvf4_pair(tmem_base, adesc + 2 * ks, bdesc + 2 * ks, idesc, (kt | ks) != 0,
-                                      sf_col + 4 * ks, sf_col + 16 + 8 * ks);
+                    // frees the stage in both CTAs and, for their scale warps, the slot
                     mma_commit_pair(&empty[stage], 0x3);
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1;
+                    if (++stage == STAGES) stage = 0;
+                    if (++slot == SF_SLOTS) {
+                        slot = 0;
+                        slot_phase ^= 1;
                     }
                 }
-                mma_commit_pair(tmem_full, 0x3);
-                acc_phase ^= 1;
+                mma_commit_pair(&acc_full[b], 0x3);
             }
             if (!ok) {
                 mma_commit_pair(drain, 0x1);
@@ -558,63 +648,127 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
             }
         }
         __syncwarp();
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ scale staging (both CTAs)
+        // The slot of stage k was last read by the MMAs of stage k - SF_SLOTS,
+        // whose completion the even CTA commits to this CTA's empty barrier.
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        int stage = 0, slot = 0;
+        uint32_t phase = 0;
+        long long kglob = 0;
+        bool ok = true;
+        for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+            for (int kt = 0; kt < p.k_tiles; ++kt, ++kglob) {
+                const long long kprev = kglob - SF_SLOTS;
+                if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull) ||
+                    (kprev >= 0 && !mbar_wait(&empty[kprev % STAGES], (uint32_t)((kprev / STAGES) & 1),
+                                              kStatusTimeoutFull))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE + lane * 16;
+                const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE + lane * 16;
+                uint32_t ra[16], rb[16], rc[16];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + ks * 512);
+                    ra[4 * ks] = a.x;
+                    ra[4 * ks + 1] = a.y;
+                    ra[4 * ks + 2] = a.z;
+                    ra[4 * ks + 3] = a.w;
+                    const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + ks * 512);
+                    const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + ks * 512);
+                    uint32_t* d = ks < 2 ? rb : rc;
+                    const int o = (ks & 1) * 8;
+                    d[o] = b0.x;
+                    d[o + 1] = b0.y;
+                    d[o + 2] = b0.z;
+                    d[o + 3] = b0.w;
+                    d[o + 4] = b1.x;
+                    d[o + 5] = b1.y;
+                    d[o + 6] = b1.z;
+                    d[o + 7] = b1.w;
+                }
+                const uint32_t col = tmem_base + lane_base + SF_COL + slot * SF_SLOT;
+                tmem_st_32x32b_x16(col, ra);
+                tmem_st_32x32b_x16(col + 16, rb);
+                tmem_st_32x32b_x16(col + 32, rc);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&sf_ready[slot]), 0));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+                if (++slot == SF_SLOTS) slot = 0;
+            }
+        }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - 4;
         const int quad = warp & 3;
         const int half = ew >> 2;
-        const uint32_t empty0 = map_shared_rank(smem_u32(tmem_empty), 0);
-        uint32_t acc_phase = 0;
         const float s_ga = *p.act_scale;
-        for (int tile = pair; tile < num_tiles; tile += npairs) {
+        const uint32_t ovl0 = map_shared_rank(smem_u32(ovl_free), 0);
+        int i = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs, ++i) {
+            const int b = i & 1;
             const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
-            if (!mbar_wait(tmem_full, acc_phase, kStatusTimeoutAccum)) break;
+            if (!mbar_wait(&acc_full[b], (i >> 1) & 1, kStatusTimeoutAccum)) break;
             tc_fence_after();
-            const int row = mb * 2 * CTA_ROWS + (int)rank * CTA_ROWS + quad * 32 + lane;
+            const int row0 = mb * 2 * CTA_ROWS + (int)rank * CTA_ROWS + quad * 32;
+            const int row = row0 + lane;
             const int ncol0 = nb * BN + half * 128;
-            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + half * 128;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (b ? ACC1_COL : 0) + half * 128;
+            using OV = Overlap<ACC1_COL>;
+            const int ov_rot = OV::rot(b, half), ov_count = OV::count(b, half);
             if (!p.out_fp32) {
                 uint32_t packed[4][16];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(taddr + j * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = ncol0 + j * 32 + h * 16;
-                        const float alpha = __fmul_rn(s_ga, segment_scale(p.segs, col < p.n ? col : p.n - 1));
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            packed[j][h * 8 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[h * 16 + 2 * e]), alpha),
-                                                               __fmul_rn(__uint_as_float(v[h * 16 + 2 * e + 1]), alpha));
-                    }
-                }
+                drain_bf16_plan<ACC1_COL>(b, half, taddr, ncol0, s_ga, p, [&] { mbar_arrive_remote(ovl0); }, lane,
+                                          packed);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty0);
-                if (row < p.m) {
-                    __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
+                if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[b]), 0));
+                uint8_t* cbuf = smem + OFF_C + ew * C_WARP;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < 4; ++j) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int col = ncol0 + j * 32 + g * 8;
-                            if (col < p.n)
-                                *reinterpret_cast<uint4*>(crow + col) =
-                                    make_uint4(packed[j][4 * g], packed[j][4 * g + 1], packed[j][4 * g + 2],
-                                               packed[j][4 * g + 3]);
+                    for (int hr = 0; hr < 2; ++hr) {
+                        if (lane == 0) bulk_wait_group_read<0>();
+                        __syncwarp();
+                        if ((lane >> 4) == hr) {
+                            const int r = lane & 15;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                *reinterpret_cast<uint4*>(cbuf + r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) =
+                                    make_uint4(packed[j][4 * u], packed[j][4 * u + 1], packed[j][4 * u + 2],
+                                               packed[j][4 * u + 3]);
                         }
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0 && row0 + 16 * hr < p.m && ncol0 + j * 32 < p.n) {
+                            tma_store_2d(&tmap_c, cbuf, ncol0 + j * 32, row0 + 16 * hr);
+                            bulk_commit_group();
+                        }
+                    }
                 }
             } else {
-                for (int j = 0; j < 4; ++j) {
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = (ov_rot + jj) & 3;
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(taddr + j * 32, v);
                     tmem_ld_wait();
-                    if (j == 3) {
+                    if (jj + 1 == ov_count) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(empty0);
+                        if (lane == 0) mbar_arrive_remote(ovl0);
+                    }
+                    if (jj == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[b]), 0));
                     }
                     const int col0 = ncol0 + j * 32;
                     if (row < p.m && col0 < p.n) {
@@ -632,10 +786,13 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
                     }
                 }
             }
-            acc_phase ^= 1;
         }
     }
 
+    if (warp >= 4 && warp < 12) {
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
     // Neither CTA leaves (or frees TMEM) while the other may still signal it.
     tc_fence_before();
     cluster_arrive_release();

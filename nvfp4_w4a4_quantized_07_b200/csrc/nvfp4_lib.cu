@@ -141,25 +141,6 @@ nvfp4_status encode_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64
     return NVFP4_OK;
 }
 
-// Tiled scale buffer viewed as 32-bit words: dim 0 = the 128 words of one
-// 512-byte atom, dim 1 = K-atoms, dim 2 = 128-row blocks.  A box of
-// {128, 4, box_blocks} is one pipeline stage's scales; atoms past the end of
-// either dimension are zero-filled by the copy engine.
-nvfp4_status encode_sf_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t k, int box_blocks)
-{
-    const int64_t katoms = pad_to(k / 16, 4) / 4;
-    const int64_t blocks = (rows + 127) / 128;
-    const cuuint64_t dims[3] = {128u, (cuuint64_t)katoms, (cuuint64_t)blocks};
-    const cuuint64_t strides[2] = {512u, (cuuint64_t)(katoms * 512)};
-    const cuuint32_t box[3] = {128u, 4u, (cuuint32_t)box_blocks};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
-    return NVFP4_OK;
-}
-
 // ---------------------------------------------------------------------------
 // Quantisation launch shared by the activation and weight entry points.
 // ---------------------------------------------------------------------------
@@ -476,7 +457,14 @@ nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int64_t m, in
         NVFP4_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(unsigned int), s));
         if ((st = launch_quant(p, s, kAmaxSiluMul, &sp, static_cast<unsigned int*>(workspace))) != NVFP4_OK)
             return st;
-        sp.h = nullptr;
+        if (h_out != nullptr) {
+            // pass 2 quantises the stored h: silu is evaluated once per element
+            p.x = h_out;
+            p.ldx = ldh;
+            p.in_fp32 = 0;
+            if ((st = launch_quant(p, s)) != NVFP4_OK) return st;
+            return ok();
+        }
     }
     if ((st = launch_quant(p, s, kQuantSiluMul, &sp)) != NVFP4_OK) return st;
     return ok();
@@ -618,11 +606,10 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         // NVFP4_GEMM_FORCE_LARGE_PAIR: CTA pairs, 256 x 256 tiles, one pair per two SMs.
         p.m_tiles = (int)((m + 255) / 256);
         p.n_tiles = (int)((n + pairk::BN - 1) / pairk::BN);
-        CUtensorMap tsa, tsw;
         if ((st = encode_fp4_map(&ta, a_q, m, k, pairk::CTA_ROWS)) != NVFP4_OK) return st;
         if ((st = encode_fp4_map(&tw, w_q, n, k, pairk::BN / 2)) != NVFP4_OK) return st;
-        if ((st = encode_sf_map(&tsa, a_sf, m, k, 1)) != NVFP4_OK) return st;
-        if ((st = encode_sf_map(&tsw, w_sf, n, k, 2)) != NVFP4_OK) return st;
+        CUtensorMap tc;
+        if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         const int pairs = (int)(tiles < dev->sms / 2 ? tiles : dev->sms / 2);
         cudaLaunchConfig_t cfg = {};
@@ -637,7 +624,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tw, tsa, tsw, p));
+        NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tw, tc, p));
         return ok();
     }
 

@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA / bulk copies,
-// tcgen05 (TMEM allocation, block-scaled MMA, SMEM->TMEM copy, TMEM loads)
-// and cluster shared memory.  Written from the PTX ISA's instruction
+// tcgen05 (TMEM allocation, block-scaled MMA, TMEM loads and stores), cluster
+// barriers and TMA stores.  Written from the PTX ISA's instruction
 // descriptions; every wait on an mbarrier is bounded.
 #pragma once
 
@@ -18,7 +18,7 @@ enum : uint32_t {
     kStatusTimeoutFull = 1u << 0,      // consumer waited too long for a TMA stage
     kStatusTimeoutEmpty = 1u << 1,     // producer waited too long for a free stage
     kStatusTimeoutAccum = 1u << 2,     // MMA / epilogue accumulator hand-off
-    kStatusTimeoutCluster = 1u << 3,   // split-K cluster reduction
+    kStatusTimeoutCluster = 1u << 3,   // decode: another CTA's partial tile never published
     kStatusTimeoutSelftest = 1u << 4,  // the deliberate self-test wait
     kStatusTimeoutDrain = 1u << 5,     // waiting for in-flight copies after an abort
 };
@@ -118,7 +118,7 @@ __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map)
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy
-// (tcgen05.cp / MMA operand reads).
+// (MMA operand reads, TMA stores).
 __device__ __forceinline__ void fence_proxy_async_shared()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -173,13 +173,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
-}
-
-// Copy a 32-row x 16-byte shared-memory matrix into TMEM, replicated into all
-// four 32-lane quadrants (the layout block-scaled MMAs read scales from).
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Each thread of the warp reads 32 consecutive 32-bit columns of its lane.
@@ -249,12 +242,6 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(const void* tile)
     return smem_desc(smem_u32(tile), 0, 1024, 2);
 }
 
-// 32 rows x 16 bytes, no swizzle: the source of tcgen05.cp.32x128b.
-__device__ __forceinline__ uint64_t desc_sf_atom(const void* atom)
-{
-    return smem_desc(smem_u32(atom), 0, 128, 0);
-}
-
 // Instruction descriptor of kind::mxf4nvf4: E2M1 A and B (format code 1),
 // UE4M3 scales, both operands K-major, FP32 accumulation, shape M x N (x 64).
 __host__ __device__ constexpr uint32_t idesc_nvf4(uint32_t m, uint32_t n)
@@ -289,32 +276,10 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t ran
     return r;
 }
 
-__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint32_t elect_one()
-{
-    uint32_t pred = 0;
-    asm volatile(
-        "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
-        "elect.sync rx|px, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, px;\n\t}"
-        : "=r"(pred));
-    return pred;
-}
-
-
 // ---------------------------------------------------------------------------
 // CTA-pair (cta_group::2) forms: two CTAs of a cluster drive one MMA of
-// M = 256.  The even CTA (rank 0) issues MMAs and TMEM copies for both; each
-// CTA keeps its own half of A, its own half of B and its own accumulator rows.
+// M = 256.  The even CTA (rank 0) issues the MMAs for both; each CTA keeps
+// its own half of A, its own half of B, its scales and its accumulator rows.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols)
 {
@@ -356,38 +321,13 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// Tiled TMA load into this CTA's shared memory whose completion is counted on
-// an mbarrier that may live in the peer CTA (a shared::cluster address).
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
-                                                 int y)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(bar_cluster)
-        : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
-                                                 int y, int z)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
-        : "memory");
-}
-
 // Arrive on an mbarrier given by its shared::cluster address (possibly in the
-// peer CTA), with release semantics at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
+// peer CTA).  Release at CTA scope, as for a local arrival: what the waiter
+// needs ordered before it are this thread's completed tcgen05 operations
+// (waited for and fenced before the arrival), not global-memory writes.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 
