@@ -50,6 +50,8 @@ def parse():
                     help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
     ap.add_argument("--probe-peaks", action="store_true",
                     help="measure the dense FP4 tensor-core rate and the HBM read rate with the probe kernels")
+    ap.add_argument("--fused", action="store_true",
+                    help="with --decode-case: time nvfp4_linear_decode (quantisation fused in)")
     ap.add_argument("--decode-case", default=None,
                     help="time one decode GEMM only, e.g. m16_5120x5120 (for ncu captures)")
     return ap.parse_args()
@@ -288,6 +290,8 @@ def run_ours(args):
     total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    qs = sorted(step_ms)
+    pct = {"p10": qs[int(0.1 * (len(qs) - 1))], "p50": statistics.median(qs), "p90": qs[int(0.9 * (len(qs) - 1))]}
 
     peaks, peak_kind = measured_peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops"]              # dense FP4 = 4 x dense BF16 (nominal ratio)
@@ -312,7 +316,8 @@ def run_ours(args):
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "step_ms_percentiles": pct,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3, fp32 accumulate), bf16 in/out",
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "m": p.m, "n": p.n, "k": p.k, "segments": p.widths,
@@ -412,10 +417,27 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
                 ms = statistics.median(times)
                 nbytes = fwd.n * k // 2 + fwd.n * k // 16 + m * k // 2 + m * k // 16 + m * fwd.n * 2
                 gbs = nbytes / (ms * 1e-3) / 1e9
+                # the whole layer in one launch: quantisation fused into the decode GEMM
+                ltimes = []
+                for it in range(13):
+                    flush.zero_()
+                    torch.cuda._sleep(400_000)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    nv.linear_decode(a, fwd, act_scale=act_scale, out=cd)
+                    e1.record(stream)
+                    torch.cuda.synchronize(device)
+                    if it >= 3:
+                        ltimes.append(e0.elapsed_time(e1))
+                lms = statistics.median(ltimes)
+                lbytes = fwd.n * k // 2 + fwd.n * k // 16 + m * k * 2 + m * fwd.n * 2
                 dec[f"m{m}_{shape}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                                        "frac_8TBs": gbs / 8000.0}
+                                        "frac_8TBs": gbs / 8000.0, "layer_us": lms * 1e3,
+                                        "layer_GB/s": lbytes / (lms * 1e-3) / 1e9}
             del fwd
         out["decode"] = {"unit": "GB/s", "bytes": "W_q + W_sf + A_q + A_sf + C (bf16), L2 flushed",
+                         "layer": "nvfp4_linear_decode: bf16 A quantised inside the GEMM, static scale; "
+                                  "bytes W_q + W_sf + A (bf16) + C (bf16)",
                          "shapes": dec}
     if not args.no_mlp:
         out.update(prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks))
@@ -585,7 +607,8 @@ def run_decode_case(args):
     device = torch.device("cuda", 0)
     p = synthetic.decode(m, shape)
     fw = nv.quantize_weight([w.to(device) for w in p.modules])
-    aq = nv.quantize_act(p.a.to(device))
+    a_dev = p.a.to(device)
+    aq = nv.quantize_act(a_dev)
     c = torch.empty((m, fw.n), dtype=torch.bfloat16, device=device)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
@@ -595,15 +618,18 @@ def run_decode_case(args):
         torch.cuda._sleep(400_000)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        nv.gemm(aq, fw, out=c)
+        if args.fused:
+            nv.linear_decode(a_dev, fw, act_scale=aq.scale, out=c)
+        else:
+            nv.gemm(aq, fw, out=c)
         e1.record(stream)
         torch.cuda.synchronize(device)
         if it >= args.warmup:
             times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
     nbytes = fw.n * p.k // 2 + fw.n * p.k // 16 + m * p.k // 2 + m * p.k // 16 + m * fw.n * 2
-    print(json.dumps({"decode_case": args.decode_case, "us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9,
-                      "steps": args.steps}), flush=True)
+    print(json.dumps({"decode_case": args.decode_case, "fused": bool(args.fused), "us": ms * 1e3,
+                      "GB/s": nbytes / (ms * 1e-3) / 1e9, "steps": args.steps}), flush=True)
     return 0
 
 

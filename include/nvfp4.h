@@ -190,6 +190,31 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_linear_decode - one W4A4 linear layer for m <= 64 tokens in a single
+ * launch: the activations are quantised to NVFP4 on the fly inside the
+ * decode GEMM (each CTA quantises the slices of A its k-range needs) and
+ * multiplied with the fused NVFP4 weight, with the per-segment scale
+ * epilogue ("Why Gated DeltaNet Survives 4-Bit Quantization": W4A4 with
+ * on-the-fly activation quantisation, abstract; per-module global scales,
+ * abstract, last sentence).  The result is bit-identical to
+ * nvfp4_quantize_act followed by nvfp4_gemm with NVFP4_GEMM_FORCE_DECODE.
+ *
+ *   a, dt, m, k, lda  raw activations as for nvfp4_quantize_act; 1 <= m <= 64
+ *                     (m == 0 is a no-op, m > 64 returns UNSUPPORTED).
+ *   act_scale_dev     device FP32 decode scale (static), or NULL: dynamic,
+ *                     amax/2688 computed inside the kernel (every CTA reads
+ *                     the whole of A, m x k, for it).
+ *   act_scale_out_dev optional device float receiving the scale used.
+ *   w_q, w_sf, n, segs, nsegs, c, odt, ldc   as for nvfp4_gemm.
+ *   workspace         device, >= nvfp4_gemm_workspace_size(m, n, k,
+ *                     NVFP4_GEMM_FORCE_DECODE) bytes, as for nvfp4_gemm.
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                 const float* act_scale_dev, float* act_scale_out_dev, const uint8_t* w_q,
+                                 const uint8_t* w_sf, int64_t n, const nvfp4_segment* segs, int nsegs, void* c,
+                                 nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_silu_mul_quantize - the glue of a gated (SwiGLU) MLP whose gate/up
  * and down projections both run as W4A4 NVFP4 GEMMs: from the BF16 gate g and
  * up u halves of the fused gate/up GEMM output it forms

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: 
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
             "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
-            "nvfp4_gemm_decode_noalloc",
+            "nvfp4_linear_decode", "nvfp4_gemm_decode_noalloc",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
 NVFP4_NOALLOC_MAX_M = 16
@@ -72,6 +72,9 @@ def load():
     L.nvfp4_silu_mul_quantize.restype = INT
     L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
     L.nvfp4_gemm.restype = INT
+    L.nvfp4_linear_decode.argtypes = [P, INT, I64, I64, I64, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P, INT,
+                                      I64, P, SZ, P]
+    L.nvfp4_linear_decode.restype = INT
     L.nvfp4_gemm_decode_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64,
                                             P]
     L.nvfp4_gemm_decode_noalloc.restype = INT
@@ -303,6 +306,32 @@ def gemm_decode_noalloc(a: QuantizedActivation, w: FusedWeight, out, segments=No
     _check("nvfp4_gemm_decode_noalloc", load().nvfp4_gemm_decode_noalloc(
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
         _ptr(out), odt, out.stride(0), _stream(out.device)))
+    return out
+
+
+def linear_decode(a, w: FusedWeight, act_scale=None, out_dtype=None, out=None, workspace=None, scale_out=None):
+    """``nvfp4_linear_decode``: one W4A4 layer for m <= 64 tokens in one launch
+    (activation quantisation fused into the decode GEMM).  ``act_scale``: a
+    1-element FP32 device scale, or ``None`` for the dynamic scale (written to
+    ``scale_out`` when given).  Returns the m x n output."""
+    import torch
+    _require_cuda(a, act_scale)
+    if a.dim() != 2 or a.stride(1) != 1:
+        raise ValueError("activations must be a 2-D tensor with unit column stride")
+    m, k = a.shape
+    if k != w.k:
+        raise ValueError("K mismatch between activations and weight")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((m, w.n), dtype=out_dtype, device=a.device)
+    odt = {torch.bfloat16: NVFP4_OUT_BF16, torch.float32: NVFP4_OUT_FP32}[out.dtype]
+    if workspace is None:
+        workspace = gemm_workspace(max(m, 1), w.n, w.k, NVFP4_GEMM_FORCE_DECODE, out.device)
+    arr = segment_array(w.segments)
+    _check("nvfp4_linear_decode", load().nvfp4_linear_decode(
+        _ptr(a), _in_dtype(a), m, k, a.stride(0), _ptr(act_scale), _ptr(scale_out), _ptr(w.q), _ptr(w.sf), w.n,
+        arr, len(w.segments), _ptr(out), odt, out.stride(0), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(out.device)))
     return out
 
 

@@ -58,6 +58,13 @@ struct GemmParams {
     int units, ctas;
     uint8_t* ws;                // [256] uint64 flags, then [256][BT][256] FP32 partial tiles
     unsigned long long epoch;   // this call's flag value
+    // decode kernel with the activation quantisation fused in: the raw
+    // activations (act_scale == nullptr: dynamic scale amax/2688, computed by
+    // every CTA; CTA 0 writes it to act_scale_out when that is given)
+    const void* a_in;
+    int64_t lda;
+    int a_fp32;
+    float* act_scale_out;
 };
 
 __device__ __forceinline__ float segment_scale(const SegTable& t, int col)

@@ -3,6 +3,7 @@
 #pragma once
 
 #include "gemm_common.cuh"
+#include "quant.cuh"
 
 namespace nvfp4 {
 
@@ -56,10 +57,10 @@ struct Cfg {
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
     static constexpr int OFF_ACC = OFF_SFB + STAGES * SFB_STAGE;
     static constexpr int OFF_BAR = OFF_ACC + BT * ACC_PITCH * 4;
-    // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full, acc_empty, drain
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 3;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, acc_full verdict, peer-wait verdict
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full, acc_empty, drain, sga_ready
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 4;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, verdicts, s_ga, amax partials
+    static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
     static_assert(A_STAGE % 1024 == 0, "SW128 stages are 1 KB aligned");
     static_assert(OFF_A + (STAGES - 1) * A_STAGE + 128 * BK_BYTES <= OFF_MISC, "MMA A reads stay in the buffer");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -99,7 +100,12 @@ __device__ __forceinline__ void store4_scaled(const GemmParams& p, int row, int 
             make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
 }
 
-template <int BT>
+// FQ: the activation quantisation is fused in.  Warps 2 and 3 then quantise
+// the stage's BT x 256 slice of the raw activations straight into the A stage
+// (the 128-byte-swizzled layout the TMA would have written) and the scale
+// atoms into the scale stage, with the same block arithmetic as
+// quantize_kernel, so the result is bit-identical to quantising first.
+template <int BT, bool FQ>
 __global__ void __launch_bounds__(decode::THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                        const __grid_constant__ GemmParams p)
@@ -118,9 +124,13 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
     uint64_t* acc_full = sf_free + SF_SLOTS;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* drain = acc_empty + 1;
+    uint64_t* sga_ready = drain + 1;   // FQ: the activation scale is in s_ga_smem
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* acc_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);    // acc_full verdict
     volatile int* peers_bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8); // a peer wait ran out
+    volatile float* s_ga_smem = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 12); // FQ: the scale used
+    volatile float* amax_part = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 16); // FQ: [2]
+    volatile int* sga_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 24);         // FQ: sga_ready verdict
     float* acc_stage = reinterpret_cast<float*>(smem + C::OFF_ACC);
 
     const int warp = threadIdx.x >> 5;
@@ -134,7 +144,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         prefetch_tensor_map(&tmap_a);
         prefetch_tensor_map(&tmap_w);
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], FQ ? 3 : 1);    // FQ: the producer and the two quantiser warps
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < SF_SLOTS; ++i) {
@@ -144,6 +154,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4);
         mbar_init(drain, 1);
+        mbar_init(sga_ready, 1);
         *peers_bad = 0;
         *acc_ok = 0;
         fence_mbarrier_init();
@@ -172,11 +183,15 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                 const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
                 const uint32_t sf_bytes = (uint32_t)nks * 512u;
                 const bool rb1 = 2 * nb + 1 < p.w_rowblocks;
-                mbar_arrive_expect_tx(&full[stage], BT * BK_BYTES + B_STAGE + sf_bytes * (rb1 ? 3u : 2u));
-                tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES, 0);
+                if (FQ) {
+                    mbar_arrive_expect_tx(&full[stage], B_STAGE + sf_bytes * (rb1 ? 2u : 1u));
+                } else {
+                    mbar_arrive_expect_tx(&full[stage], BT * BK_BYTES + B_STAGE + sf_bytes * (rb1 ? 3u : 2u));
+                    tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES, 0);
+                    bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_sf + (int64_t)kt * KSTEPS * 512, sf_bytes,
+                              &full[stage]);
+                }
                 tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, nb * BN);
-                bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_sf + (int64_t)kt * KSTEPS * 512, sf_bytes,
-                          &full[stage]);
                 bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
                           p.w_sf + ((int64_t)(2 * nb) * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
                 if (rb1)
@@ -249,6 +264,90 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
             }
         }
         __syncwarp();
+    } else if (FQ && (warp == 2 || warp == 3)) {
+        // ------------------------------------------------------------ activation quantiser
+        const int qt = threadIdx.x - 64;    // 0..63
+        float s_ga;
+        if (p.act_scale != nullptr) {
+            s_ga = *p.act_scale;
+        } else {
+            // amax over the whole m x k activation (every CTA computes the same, exact value)
+            const int vec = p.a_fp32 ? 4 : 8;
+            const int64_t per_row = p.k / vec;
+            const int64_t total = (int64_t)p.m * per_row;
+            float mx = 0.0f;
+            for (int64_t i = qt; i < total; i += 64) {
+                const int64_t r = i / per_row;
+                mx = fmaxf(mx, absmax_vec(p.a_in, r * p.lda + (i - r * per_row) * vec, p.a_fp32));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) amax_part[warp - 2] = mx;
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            s_ga = global_scale_from_amax(fmaxf(amax_part[0], amax_part[1]));
+        }
+        if (qt == 0) {
+            *s_ga_smem = s_ga;
+            mbar_arrive(sga_ready);
+            if (cta == 0 && p.act_scale_out != nullptr) *p.act_scale_out = s_ga;
+        }
+        int stage = 0;
+        uint32_t phase = 0;
+        int kt = (int)(u_begin % k_tiles);
+        const int64_t esz = p.a_fp32 ? 4 : 2;
+        for (int64_t u = u_begin; u < u_end; ++u) {
+            if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) break;
+            uint8_t* adst = smem + OFF_A + stage * A_STAGE;
+            uint8_t* sdst = smem + OFF_SFA + stage * SFA_STAGE;
+            for (int it = qt; it < BT * 8; it += 64) {
+                // row r, 32-element chunk c of this 256-deep k-tile: two 16-element blocks
+                const int r = it >> 3, c = it & 7;
+                const int64_t k0 = (int64_t)kt * 256 + c * 32;
+                const bool live0 = r < p.m && k0 < p.k;
+                const bool live1 = r < p.m && k0 + 16 < p.k;
+                float v0[16], v1[16];
+                const uint8_t* src = static_cast<const uint8_t*>(p.a_in) + ((int64_t)r * p.lda + k0) * esz;
+                if (p.a_fp32) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 f0 = live0 ? __ldg(reinterpret_cast<const float4*>(src) + j)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                        const float4 f1 = live1 ? __ldg(reinterpret_cast<const float4*>(src) + 4 + j)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                        v0[4 * j] = f0.x; v0[4 * j + 1] = f0.y; v0[4 * j + 2] = f0.z; v0[4 * j + 3] = f0.w;
+                        v1[4 * j] = f1.x; v1[4 * j + 1] = f1.y; v1[4 * j + 2] = f1.z; v1[4 * j + 3] = f1.w;
+                    }
+                } else {
+                    uint4 w[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        w[j] = ((j < 2) ? live0 : live1) ? __ldg(reinterpret_cast<const uint4*>(src) + j)
+                                                         : make_uint4(0, 0, 0, 0);
+                    unpack_bf16x8(w[0], v0);
+                    unpack_bf16x8(w[1], v0 + 8);
+                    unpack_bf16x8(w[2], v1);
+                    unpack_bf16x8(w[3], v1 + 8);
+                }
+                uint32_t sb0, sb1;
+                uint2 q0, q1;
+                quantize_block16(v0, s_ga, live0, sb0, q0);
+                quantize_block16(v1, s_ga, live1, sb1, q1);
+                // K-major 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+                *reinterpret_cast<uint4*>(adst + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(q0.x, q0.y, q1.x, q1.y);
+                // scale atom of k-step c / 2: row r at (r % 32) * 16 + (r / 32 % 4) * 4, block (c % 2) * 2
+                *reinterpret_cast<uint16_t*>(sdst + (c >> 1) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
+                                             (c & 1) * 2) = (uint16_t)(sb0 | (sb1 << 8));
+            }
+            fence_proxy_async_shared();     // the MMA reads the stage through the async proxy
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1;
+            }
+            if (++kt == k_tiles) kt = 0;
+        }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ scale staging
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -318,7 +417,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         const bool live = quad * 32 < BT;          // warp holds loaded token rows
         unsigned long long* flags = reinterpret_cast<unsigned long long*>(p.ws);
         float* parts = reinterpret_cast<float*>(p.ws + FLAGS_BYTES);
-        const float s_ga = *p.act_scale;
+        float s_ga = FQ ? 0.0f : *p.act_scale;        // FQ: known once the first stage is in
         const int units4 = min(p.m, BT) * (BN / 4);  // float4 units of the live rows
         uint32_t segs = 0;
         int64_t u = u_begin;
@@ -332,6 +431,15 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
             if (et == 0) *acc_ok = mbar_wait(acc_full, segs & 1, kStatusTimeoutAccum) ? 1 : 0;
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!*acc_ok) break;
+            if (FQ && segs == 0) {
+                // bounded like every wait; the quantiser set it before its first stage
+                if (et == 0) *sga_ok = mbar_wait(sga_ready, 0, kStatusTimeoutAccum) ? 1 : 0;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (!*sga_ok) break;
+                s_ga = *s_ga_smem;
+            } else if (FQ) {
+                s_ga = *s_ga_smem;
+            }
             tc_fence_after();
             if (live) {
                 const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
@@ -422,7 +530,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                 const int last = cta_of_unit((int64_t)(nb + 1) * k_tiles - 1, p.units, p.ctas);
                 const int units4 = min(p.m, BT) * (BN / 4);
                 const float* parts = reinterpret_cast<const float*>(p.ws + FLAGS_BYTES);
-                const float s_ga = *p.act_scale;
+                const float s_ga = FQ ? *s_ga_smem : *p.act_scale;
                 for (int x0 = threadIdx.x; x0 < units4; x0 += FDU * THREADS) {
                     float4 v[FDU];
 #pragma unroll

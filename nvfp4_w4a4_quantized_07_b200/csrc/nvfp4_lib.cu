@@ -82,12 +82,18 @@ nvfp4_status device_state(DeviceState** out)
                                             large::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             pairk::SMEM_BYTES));
-        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Cfg<16>::SMEM_BYTES));
-        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Cfg<32>::SMEM_BYTES));
-        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            decode::Cfg<64>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<16>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<16>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<32>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<32, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<32>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<64, false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<64>::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<64, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, decode::Cfg<64>::SMEM_BYTES));
         d.ready = true;
     }
     *out = &d;
@@ -277,7 +283,7 @@ unsigned long long next_epoch()
     return g_epoch.fetch_add(2ull) + 2ull;
 }
 
-template <int BT>
+template <int BT, bool FQ>
 nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& p, cudaStream_t s)
 {
     cudaLaunchConfig_t cfg = {};
@@ -292,7 +298,7 @@ nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, const G
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT>, ta, tw, p));
+    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT, FQ>, ta, tw, p));
     return NVFP4_OK;
 }
 
@@ -642,9 +648,81 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     p.n_tiles = w_tiles;
     if ((st = encode_fp4_map(&ta, a_q, m, k, bt)) != NVFP4_OK) return st;
     if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
-    if (bt == 16) st = launch_decode<16>(ta, tw, p, s);
-    else if (bt == 32) st = launch_decode<32>(ta, tw, p, s);
-    else st = launch_decode<64>(ta, tw, p, s);
+    if (bt == 16) st = launch_decode<16, false>(ta, tw, p, s);
+    else if (bt == 32) st = launch_decode<32, false>(ta, tw, p, s);
+    else st = launch_decode<64, false>(ta, tw, p, s);
+    if (st != NVFP4_OK) return st;
+    return ok();
+}
+
+nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                 const float* act_scale_dev, float* act_scale_out_dev, const uint8_t* w_q,
+                                 const uint8_t* w_sf, int64_t n, const nvfp4_segment* segs, int nsegs, void* c,
+                                 nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, void* stream)
+{
+    nvfp4_status st = check_quant_input(a, dt, m, k, lda, "linear_decode");
+    if (st != NVFP4_OK) return st;
+    if (m > 64) return fail(NVFP4_ERR_UNSUPPORTED, "linear_decode: m = %lld > 64 (use nvfp4_quantize_act + nvfp4_gemm)",
+                            (long long)m);
+    if (n <= 0 || n % 16 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_decode: n must be a positive multiple of 16 (n=%lld)", (long long)n);
+    if (n >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "linear_decode: dimension >= 2^31");
+    if (odt != NVFP4_OUT_BF16 && odt != NVFP4_OUT_FP32)
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_decode: bad output dtype");
+    if (ldc < n) return fail(NVFP4_ERR_INVALID_ARG, "linear_decode: ldc %lld < n %lld", (long long)ldc, (long long)n);
+    SegTable table;
+    if ((st = check_segments(segs, nsegs, n, &table)) != NVFP4_OK) return st;
+    if (m > 0 && (w_q == nullptr || w_sf == nullptr || c == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_decode: NULL weight or output pointer");
+    const int64_t osz = odt == NVFP4_OUT_FP32 ? 4 : 2;
+    if (!aligned16(w_q) || !aligned16(w_sf) || !aligned16(c) || (ldc * osz) % 16 != 0)
+        return fail(NVFP4_ERR_ALIGNMENT, "linear_decode: weights and output rows must be 16-byte aligned");
+    if (workspace == nullptr || ws_bytes < decode_ws_bytes(m < 1 ? 1 : m))
+        return fail(NVFP4_ERR_WORKSPACE, "linear_decode: needs %zu bytes of workspace (got %zu)",
+                    decode_ws_bytes(m < 1 ? 1 : m), ws_bytes);
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "linear_decode: workspace not 16-byte aligned");
+    if (m == 0) return ok();
+
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GemmParams p = {};
+    p.m = (int)m;
+    p.n = (int)n;
+    p.k = (int)k;
+    p.w_sf = w_sf;
+    p.act_scale = act_scale_dev;
+    p.c = c;
+    p.ldc = ldc;
+    p.out_fp32 = odt == NVFP4_OUT_FP32;
+    p.segs = table;
+    p.katoms = (int)(pad_to(k / 16, 4) / 4);
+    p.k_tiles = (int)((k + 255) / 256);
+    p.a_rowblocks = 1;
+    p.w_rowblocks = (int)((n + 127) / 128);
+    p.splits = 1;
+    p.a_in = a;
+    p.lda = lda;
+    p.a_fp32 = dt == NVFP4_IN_FP32;
+    p.act_scale_out = act_scale_out_dev;
+    const int bt = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
+    const int w_tiles = (int)((n + decode::BN - 1) / decode::BN);
+    const int64_t units = (int64_t)w_tiles * p.k_tiles;
+    if (units >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "linear_decode: problem too large");
+    int64_t ctas = dev->sms < decode::MAX_CTAS ? dev->sms : decode::MAX_CTAS;
+    if (ctas > units) ctas = units;
+    p.units = (int)units;
+    p.ctas = (int)ctas;
+    p.ws = static_cast<uint8_t*>(workspace);
+    p.epoch = next_epoch();
+    p.m_tiles = 1;
+    p.n_tiles = w_tiles;
+    CUtensorMap tw;
+    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
+    // the A map is not read when the quantisation is fused in
+    if (bt == 16) st = launch_decode<16, true>(tw, tw, p, s);
+    else if (bt == 32) st = launch_decode<32, true>(tw, tw, p, s);
+    else st = launch_decode<64, true>(tw, tw, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
 }

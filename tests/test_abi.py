@@ -194,3 +194,19 @@ def test_silu_mul_quantize_argument_errors(lib):
     assert f(FAKE, FAKE, 8, 64, 128, None, None, FAKE, FAKE, None, 0, ws, 256, None) == 1    # dynamic: no scale out
     assert f(FAKE, FAKE, 8, 64, 128, None, FAKE, FAKE, FAKE, None, 0, None, 0, None) == 6    # dynamic: no workspace
     assert f(FAKE, FAKE, 0, 64, 128, FAKE, None, FAKE, FAKE, None, 0, None, 0, None) == 0    # empty
+
+
+def test_linear_decode_argument_errors(lib):
+    f = lib.nvfp4_linear_decode
+    s = _segs((0, 64, 1.0))
+    ws = ctypes.c_void_p(0x40000)
+    need = lib.nvfp4_gemm_workspace_size(8, 64, 64, 2)
+    assert f(FAKE, 0, 65, 64, 64, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, ws, need, None) == 2   # m > 64
+    assert f(FAKE, 0, 8, 48, 48, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, ws, need, None) == 1    # k % 32
+    assert f(FAKE, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, 40, _segs((0, 40, 1.0)), 1, FAKE, 0, 40, ws, need,
+             None) == 1                                                                                  # n % 16
+    assert f(FAKE, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, None, 0, None) == 6     # workspace
+    assert f(MISALIGNED, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, ws, need, None) == 3
+    assert f(FAKE, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, 64, _segs((0, 48, 1.0)), 1, FAKE, 0, 64, ws, need,
+             None) == 1                                                                                  # segments
+    assert f(FAKE, 0, 0, 64, 64, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, ws, need, None) == 0     # empty
