@@ -190,6 +190,31 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_gemm_swiglu_quantize - the gate/up GEMM of a gated MLP with its glue
+ * fused into the epilogue: for the fused weight [gate (f rows); up (f rows)]
+ * (2f x k, e.g. two separately calibrated modules with their own segment
+ * scales) it computes, per output element j < f,
+ *     g = bf16(acc_gate * s_ga * s_gw[seg(j)]),  u = bf16(acc_up * s_ga * s_gw[seg(f + j)]),
+ *     h = bf16(silu(g) * u)
+ * and quantises h to NVFP4 with the static decode scale *h_scale_dev,
+ * writing codes and tiled scales only (h itself never reaches memory).  The
+ * bytes equal nvfp4_gemm (BF16 output) followed by nvfp4_silu_mul_quantize
+ * with the same static scale.  The pages do not describe the MLP; this is the
+ * step between its two W4A4 linear layers.
+ *
+ *   a_q, a_sf, act_scale_dev  quantised activations, m x k (as for nvfp4_gemm).
+ *   w_q, w_sf                 fused weight, 2f rows; f a multiple of 128.
+ *   segs, nsegs               segment table over the 2f columns.
+ *   h_scale_dev               device FP32 decode scale of h (calibrated).
+ *   h_q, h_sf                 outputs: m x f/2 codes, nvfp4_sf_bytes(m, f)
+ *                             tiled scale bytes (padding rows zeroed).
+ * ---------------------------------------------------------------------- */
+NVFP4_API nvfp4_status nvfp4_gemm_swiglu_quantize(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
+                                        const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t f, int64_t k,
+                                        const nvfp4_segment* segs, int nsegs, const float* h_scale_dev,
+                                        uint8_t* h_q, uint8_t* h_sf, void* stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_linear_decode - one W4A4 linear layer for m <= 64 tokens in a single
  * launch: the activations are quantised to NVFP4 on the fly inside the
  * decode GEMM (each CTA quantises the slices of A its k-range needs) and

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: 
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
             "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
-            "nvfp4_linear_decode", "nvfp4_gemm_decode_noalloc",
+            "nvfp4_linear_decode", "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
 NVFP4_NOALLOC_MAX_M = 16
@@ -72,6 +72,8 @@ def load():
     L.nvfp4_silu_mul_quantize.restype = INT
     L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
     L.nvfp4_gemm.restype = INT
+    L.nvfp4_gemm_swiglu_quantize.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, P, P, P]
+    L.nvfp4_gemm_swiglu_quantize.restype = INT
     L.nvfp4_linear_decode.argtypes = [P, INT, I64, I64, I64, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P, INT,
                                       I64, P, SZ, P]
     L.nvfp4_linear_decode.restype = INT
@@ -306,6 +308,29 @@ def gemm_decode_noalloc(a: QuantizedActivation, w: FusedWeight, out, segments=No
     _check("nvfp4_gemm_decode_noalloc", load().nvfp4_gemm_decode_noalloc(
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
         _ptr(out), odt, out.stride(0), _stream(out.device)))
+    return out
+
+
+def gemm_swiglu_quantize(a: QuantizedActivation, w: FusedWeight, h_scale, out: QuantizedActivation | None = None):
+    """``nvfp4_gemm_swiglu_quantize``: the gate/up GEMM of a gated MLP with
+    h = bf16(silu(g) * u) quantised in its epilogue (static scale ``h_scale``,
+    a 1-element FP32 device tensor).  ``w`` holds [gate; up] (2f rows).
+    Returns h as a QuantizedActivation (m x f), ready for the down GEMM."""
+    import torch
+    _require_cuda(h_scale)
+    if a.k != w.k or w.n % 2 != 0:
+        raise ValueError("K mismatch, or the weight is not [gate; up]")
+    f = w.n // 2
+    L = load()
+    if out is None:
+        out = QuantizedActivation(
+            q=torch.empty((a.m, f // 2), dtype=torch.uint8, device=a.q.device),
+            sf=torch.empty(max(L.nvfp4_sf_bytes(a.m, f), 1), dtype=torch.uint8, device=a.q.device),
+            scale=h_scale, m=a.m, k=f)
+    arr = segment_array(w.segments)
+    _check("nvfp4_gemm_swiglu_quantize", L.nvfp4_gemm_swiglu_quantize(
+        _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, f, w.k, arr, len(w.segments),
+        _ptr(h_scale), _ptr(out.q), _ptr(out.sf), _stream(a.q.device)))
     return out
 
 

@@ -65,6 +65,13 @@ struct GemmParams {
     int64_t lda;
     int a_fp32;
     float* act_scale_out;
+    // large-M kernel with the SwiGLU epilogue: the weight is [gate (f rows);
+    // up (f rows)] and the epilogue writes h = bf16(silu(g) * u) quantised
+    // with the static decode scale h_scale (codes m x f/2, tiled scales)
+    int swiglu_f;
+    const float* h_scale;
+    uint8_t* h_q;
+    uint8_t* h_sf;
 };
 
 __device__ __forceinline__ float segment_scale(const SegTable& t, int col)

@@ -295,50 +295,79 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         uint32_t phase = 0;
         int kt = (int)(u_begin % k_tiles);
         const int64_t esz = p.a_fp32 ? 4 : 2;
+        // Each thread owns BT / 8 chunks (row r, 32 columns) of a stage, taken two
+        // at a time: all loads of a pair are issued before any arithmetic, and
+        // the first pair's loads before the wait for the stage buffer (they do
+        // not need it), so the L2 round trip overlaps the wait.
+        constexpr int CPT = BT / 8;
+        constexpr int CB = CPT < 2 ? CPT : 2;
         for (int64_t u = u_begin; u < u_end; ++u) {
-            if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) break;
             uint8_t* adst = smem + OFF_A + stage * A_STAGE;
             uint8_t* sdst = smem + OFF_SFA + stage * SFA_STAGE;
-            for (int it = qt; it < BT * 8; it += 64) {
-                // row r, 32-element chunk c of this 256-deep k-tile: two 16-element blocks
-                const int r = it >> 3, c = it & 7;
-                const int64_t k0 = (int64_t)kt * 256 + c * 32;
-                const bool live0 = r < p.m && k0 < p.k;
-                const bool live1 = r < p.m && k0 + 16 < p.k;
-                float v0[16], v1[16];
-                const uint8_t* src = static_cast<const uint8_t*>(p.a_in) + ((int64_t)r * p.lda + k0) * esz;
-                if (p.a_fp32) {
+            bool waited = false, ok = true;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 f0 = live0 ? __ldg(reinterpret_cast<const float4*>(src) + j)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                        const float4 f1 = live1 ? __ldg(reinterpret_cast<const float4*>(src) + 4 + j)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                        v0[4 * j] = f0.x; v0[4 * j + 1] = f0.y; v0[4 * j + 2] = f0.z; v0[4 * j + 3] = f0.w;
-                        v1[4 * j] = f1.x; v1[4 * j + 1] = f1.y; v1[4 * j + 2] = f1.z; v1[4 * j + 3] = f1.w;
+            for (int b0 = 0; b0 < CPT; b0 += CB) {
+                uint4 raw[CB][8];
+                bool l0[CB], l1[CB];
+#pragma unroll
+                for (int j = 0; j < CB; ++j) {
+                    const int it = qt + 64 * (b0 + j);
+                    const int r = it >> 3, c = it & 7;
+                    const int64_t k0 = (int64_t)kt * 256 + c * 32;
+                    l0[j] = r < p.m && k0 < p.k;
+                    l1[j] = r < p.m && k0 + 16 < p.k;
+                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.a_in) +
+                                                                      ((int64_t)r * p.lda + k0) * esz);
+                    const int words = p.a_fp32 ? 8 : 4;   // 16-byte words per 32 elements
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const bool lv = (w < words / 2) ? l0[j] : l1[j];
+                        raw[j][w] = (w < words && lv) ? __ldg(src + w) : make_uint4(0, 0, 0, 0);
                     }
-                } else {
-                    uint4 w[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        w[j] = ((j < 2) ? live0 : live1) ? __ldg(reinterpret_cast<const uint4*>(src) + j)
-                                                         : make_uint4(0, 0, 0, 0);
-                    unpack_bf16x8(w[0], v0);
-                    unpack_bf16x8(w[1], v0 + 8);
-                    unpack_bf16x8(w[2], v1);
-                    unpack_bf16x8(w[3], v1 + 8);
                 }
-                uint32_t sb0, sb1;
-                uint2 q0, q1;
-                quantize_block16(v0, s_ga, live0, sb0, q0);
-                quantize_block16(v1, s_ga, live1, sb1, q1);
-                // K-major 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
-                *reinterpret_cast<uint4*>(adst + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-                    make_uint4(q0.x, q0.y, q1.x, q1.y);
-                // scale atom of k-step c / 2: row r at (r % 32) * 16 + (r / 32 % 4) * 4, block (c % 2) * 2
-                *reinterpret_cast<uint16_t*>(sdst + (c >> 1) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
-                                             (c & 1) * 2) = (uint16_t)(sb0 | (sb1 << 8));
+                if (!waited) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    waited = true;
+                }
+#pragma unroll
+                for (int j = 0; j < CB; ++j) {
+                    const int it = qt + 64 * (b0 + j);
+                    const int r = it >> 3, c = it & 7;
+                    float v0[16], v1[16];
+                    if (p.a_fp32) {
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            v0[4 * w] = __uint_as_float(raw[j][w].x);
+                            v0[4 * w + 1] = __uint_as_float(raw[j][w].y);
+                            v0[4 * w + 2] = __uint_as_float(raw[j][w].z);
+                            v0[4 * w + 3] = __uint_as_float(raw[j][w].w);
+                            v1[4 * w] = __uint_as_float(raw[j][4 + w].x);
+                            v1[4 * w + 1] = __uint_as_float(raw[j][4 + w].y);
+                            v1[4 * w + 2] = __uint_as_float(raw[j][4 + w].z);
+                            v1[4 * w + 3] = __uint_as_float(raw[j][4 + w].w);
+                        }
+                    } else {
+                        unpack_bf16x8(raw[j][0], v0);
+                        unpack_bf16x8(raw[j][1], v0 + 8);
+                        unpack_bf16x8(raw[j][2], v1);
+                        unpack_bf16x8(raw[j][3], v1 + 8);
+                    }
+                    uint32_t sb0, sb1;
+                    uint2 q0, q1;
+                    quantize_block16(v0, s_ga, l0[j], sb0, q0);
+                    quantize_block16(v1, s_ga, l1[j], sb1, q1);
+                    // K-major 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+                    *reinterpret_cast<uint4*>(adst + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(q0.x, q0.y, q1.x, q1.y);
+                    // scale atom of k-step c / 2: row r at (r % 32) * 16 + (r / 32 % 4) * 4, block (c % 2) * 2
+                    *reinterpret_cast<uint16_t*>(sdst + (c >> 1) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
+                                                 (c & 1) * 2) = (uint16_t)(sb0 | (sb1 << 8));
+                }
             }
+            if (!ok) break;
             fence_proxy_async_shared();     // the MMA reads the stage through the async proxy
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[stage]);

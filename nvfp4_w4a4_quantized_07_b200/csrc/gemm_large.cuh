@@ -4,6 +4,7 @@
 #pragma once
 
 #include "gemm_common.cuh"
+#include "quant.cuh"
 
 namespace nvfp4 {
 
@@ -136,6 +137,14 @@ static_assert(ACC1_COL + BN <= SF_COL && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COL
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace large
 
+// SWIGLU: the gate/up GEMM of a gated MLP with its glue fused into the
+// epilogue.  Each 128 x 256 tile holds 128 gate columns (accumulator columns
+// 0..127) and the matching 128 up columns (128..255), loaded as two 128-row
+// boxes of the [gate; up] weight; the epilogue forms
+// h = bf16(silu(bf16(g)) * bf16(u)) exactly as the unfused GEMM (BF16 output)
+// followed by silu_mul_quantize_kernel would, and quantises it with the
+// static scale h_scale, writing codes and tiled scales instead of C.
+template <bool SWIGLU>
 __global__ void __launch_bounds__(large::THREADS, 1)
     gemm_large_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ GemmParams p)
@@ -171,7 +180,8 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 8);
         }
-        mbar_init(ovl_free, Overlap<ACC1_COL>::warps());
+        // SWIGLU: every epilogue warp reads gate and up columns; all release after their drain
+        mbar_init(ovl_free, SWIGLU ? 8 : Overlap<ACC1_COL>::warps());
         mbar_init(drain, 1);
         fence_mbarrier_init();
     }
@@ -199,19 +209,27 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                     }
                     const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
                     const uint32_t sf_bytes = (uint32_t)nks * 512u;
-                    const bool w_rb1 = 2 * nb + 1 < p.w_rowblocks;
+                    // weight row blocks of the tile's two 128-row halves
+                    const int rb0 = SWIGLU ? nb : 2 * nb;
+                    const int rb1 = SWIGLU ? p.swiglu_f / 128 + nb : 2 * nb + 1;
+                    const bool w_rb1 = rb1 < p.w_rowblocks;
                     const uint32_t bytes = A_STAGE + B_STAGE + sf_bytes * (w_rb1 ? 3u : 2u);
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES, mb * BM);
-                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, nb * BN);
+                    if (SWIGLU) {
+                        tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, rb0 * 128);
+                        tma_load_2d(smem + OFF_B + stage * B_STAGE + 128 * BK_BYTES, &tmap_w, &full[stage],
+                                    kt * BK_BYTES, rb1 * 128);
+                    } else {
+                        tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, nb * BN);
+                    }
                     bulk_load(smem + OFF_SFA + stage * SFA_STAGE,
                               p.a_sf + ((int64_t)mb * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
                     bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
-                              p.w_sf + ((int64_t)(2 * nb) * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
+                              p.w_sf + ((int64_t)rb0 * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
                     if (w_rb1)
                         bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
-                                  p.w_sf + ((int64_t)(2 * nb + 1) * p.katoms + kt * KSTEPS) * 512, sf_bytes,
-                                  &full[stage]);
+                                  p.w_sf + ((int64_t)rb1 * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -369,7 +387,57 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             // and released (Overlap<ACC1_COL>).
             using OV = Overlap<ACC1_COL>;
             const int ov_rot = OV::rot(b, half), ov_count = OV::count(b, half);
-            if (!p.out_fp32) {
+            if (SWIGLU) {
+                // warp (quad, half): gate chunks 2 half, 2 half + 1 with the up
+                // chunks 4 columns-of-32 to the right; 64 h columns per row
+                const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (b ? ACC1_COL : 0);
+                const float s_h = *p.h_scale;
+                const int hcol0 = nb * 128 + half * 64;             // first h column of this warp
+                uint32_t sfw = 0;
+#pragma unroll
+                for (int g2 = 0; g2 < 2; ++g2) {
+                    const int gc = 2 * half + g2;                    // gate chunk; up chunk is gc + 4
+                    uint32_t vg[32], vu[32];
+                    tmem_ld_32x32b_x32(tacc + gc * 32, vg);
+                    tmem_ld_32x32b_x32(tacc + (gc + 4) * 32, vu);
+                    tmem_ld_wait();
+                    const int gcol = hcol0 + 32 * g2;                // gate column in the fused weight
+                    const float ag0 = __fmul_rn(s_ga, segment_scale(p.segs, gcol));
+                    const float ag1 = __fmul_rn(s_ga, segment_scale(p.segs, gcol + 16));
+                    const float au0 = __fmul_rn(s_ga, segment_scale(p.segs, p.swiglu_f + gcol));
+                    const float au1 = __fmul_rn(s_ga, segment_scale(p.segs, p.swiglu_f + gcol + 16));
+                    float h0[16], h1[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float g0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vg[e]), ag0)));
+                        const float u0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vu[e]), au0)));
+                        const float g1 =
+                            __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vg[16 + e]), ag1)));
+                        const float u1 =
+                            __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vu[16 + e]), au1)));
+                        h0[e] = silu_mul_bf16(g0, u0);
+                        h1[e] = silu_mul_bf16(g1, u1);
+                    }
+                    const bool live = row < p.m;
+                    uint32_t sb0, sb1;
+                    uint2 q0, q1;
+                    quantize_block16(h0, s_h, live, sb0, q0);
+                    quantize_block16(h1, s_h, live, sb1, q1);
+                    if (live)
+                        *reinterpret_cast<uint4*>(p.h_q + (int64_t)row * (p.swiglu_f >> 1) + (gcol >> 1)) =
+                            make_uint4(q0.x, q0.y, q1.x, q1.y);
+                    sfw |= (sb0 | (sb1 << 8)) << (16 * g2);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(ovl_free);
+                    mbar_arrive(&acc_empty[b]);
+                }
+                // four consecutive 16-column blocks of h: one word of the row's atom
+                // (zero on the padding rows, which the tiled layout requires)
+                *reinterpret_cast<uint32_t*>(p.h_sf + sf_tiled_offset(row, hcol0 >> 4, p.swiglu_f >> 6)) = sfw;
+            } else if (!p.out_fp32) {
                 uint32_t packed[4][16];
                 drain_bf16_plan<ACC1_COL>(b, half, taddr, ncol0, s_ga, p, [&] { mbar_arrive(ovl_free); }, lane,
                                           packed);

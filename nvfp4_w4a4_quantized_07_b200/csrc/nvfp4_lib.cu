@@ -78,7 +78,9 @@ nvfp4_status device_state(DeviceState** out)
             return fail(NVFP4_ERR_UNSUPPORTED, "device %d is sm_%d%d; libnvfp4 is built for sm_100a only", dev, major,
                         minor);
         NVFP4_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
-        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            large::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             large::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             pairk::SMEM_BYTES));
@@ -604,7 +606,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
-        gemm_large_kernel<<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tc, p);
+        gemm_large_kernel<false><<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tc, p);
         NVFP4_CUDA_TRY(cudaGetLastError());
         return ok();
     }
@@ -652,6 +654,60 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     else if (bt == 32) st = launch_decode<32, false>(ta, tw, p, s);
     else st = launch_decode<64, false>(ta, tw, p, s);
     if (st != NVFP4_OK) return st;
+    return ok();
+}
+
+nvfp4_status nvfp4_gemm_swiglu_quantize(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
+                                        const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t f, int64_t k,
+                                        const nvfp4_segment* segs, int nsegs, const float* h_scale_dev,
+                                        uint8_t* h_q, uint8_t* h_sf, void* stream)
+{
+    if (m < 0 || f <= 0 || f % 128 != 0 || k <= 0 || k % 32 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm_swiglu_quantize: need m >= 0, f a positive multiple of 128 and k a "
+                                           "positive multiple of 32 (m=%lld f=%lld k=%lld)",
+                    (long long)m, (long long)f, (long long)k);
+    if (m >= (1ll << 31) || 2 * f >= (1ll << 31) || k >= (1ll << 31))
+        return fail(NVFP4_ERR_UNSUPPORTED, "gemm_swiglu_quantize: dimension >= 2^31");
+    SegTable table;
+    nvfp4_status st = check_segments(segs, nsegs, 2 * f, &table);
+    if (st != NVFP4_OK) return st;
+    if (m > 0 && (a_q == nullptr || a_sf == nullptr || act_scale_dev == nullptr || w_q == nullptr ||
+                  w_sf == nullptr || h_scale_dev == nullptr || h_q == nullptr || h_sf == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm_swiglu_quantize: NULL pointer");
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(h_q) ||
+        !aligned16(h_sf))
+        return fail(NVFP4_ERR_ALIGNMENT, "gemm_swiglu_quantize: operands and outputs must be 16-byte aligned");
+    if (m == 0) return ok();
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GemmParams p = {};
+    p.m = (int)m;
+    p.n = (int)(2 * f);
+    p.k = (int)k;
+    p.a_sf = a_sf;
+    p.w_sf = w_sf;
+    p.act_scale = act_scale_dev;
+    p.segs = table;
+    p.katoms = (int)(pad_to(k / 16, 4) / 4);
+    p.k_tiles = (int)((k + 255) / 256);
+    p.a_rowblocks = (int)((m + 127) / 128);
+    p.w_rowblocks = (int)((2 * f + 127) / 128);
+    p.splits = 1;
+    p.swiglu_f = (int)f;
+    p.h_scale = h_scale_dev;
+    p.h_q = h_q;
+    p.h_sf = h_sf;
+    p.m_tiles = (int)((m + large::BM - 1) / large::BM);
+    p.n_tiles = (int)(f / 128);
+    CUtensorMap ta, tw;
+    if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
+    if ((st = encode_fp4_map(&tw, w_q, 2 * f, k, 128)) != NVFP4_OK) return st;
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
+    // no C is written: the C map argument is not read
+    gemm_large_kernel<true><<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tw, p);
+    NVFP4_CUDA_TRY(cudaGetLastError());
     return ok();
 }
 

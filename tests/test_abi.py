@@ -210,3 +210,14 @@ def test_linear_decode_argument_errors(lib):
     assert f(FAKE, 0, 8, 64, 64, FAKE, None, FAKE, FAKE, 64, _segs((0, 48, 1.0)), 1, FAKE, 0, 64, ws, need,
              None) == 1                                                                                  # segments
     assert f(FAKE, 0, 0, 64, 64, FAKE, None, FAKE, FAKE, 64, s, 1, FAKE, 0, 64, ws, need, None) == 0     # empty
+
+
+def test_gemm_swiglu_quantize_argument_errors(lib):
+    f = lib.nvfp4_gemm_swiglu_quantize
+    s2 = _segs((0, 128, 1.0), (128, 256, 1.0))
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 64, 64, _segs((0, 128, 1.0)), 1, FAKE, FAKE, FAKE, None) == 1  # f % 128
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 48, s2, 2, FAKE, FAKE, FAKE, None) == 1                    # k % 32
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, _segs((0, 128, 1.0)), 1, FAKE, FAKE, FAKE, None) == 1  # segs
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, s2, 2, None, FAKE, FAKE, None) == 1                    # no scale
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, s2, 2, FAKE, MISALIGNED, FAKE, None) == 3
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 64, s2, 2, FAKE, FAKE, FAKE, None) == 0                    # empty

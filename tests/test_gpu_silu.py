@@ -163,3 +163,32 @@ def test_config_long_prefill_mlp_sampled():
     w2_hat = oracle.dequantize(qw2, sfw2, s_w2)
     c2_s = c2[rsel][:, torch.from_numpy(pick).to(dev)]
     assert_gemm_close(c2_s, oracle.gemm(h_hat, w2_hat), h_hat, w2_hat, "down GEMM")
+
+
+FUSED_CASES = [
+    # (m, f, k)
+    (300, 256, 512),
+    (129, 1024, 1056),
+    (8192, 17408, 5120),
+]
+
+
+@pytest.mark.parametrize("m,f,k", FUSED_CASES)
+def test_swiglu_epilogue_equals_gemm_then_glue(m, f, k):
+    """nvfp4_gemm_swiglu_quantize (glue in the gate/up GEMM's epilogue, static
+    h scale) must give the bytes of the BF16 gate/up GEMM followed by
+    nvfp4_silu_mul_quantize with the same scale."""
+    a, _ = synthetic.activations(m, k, seed=m + f + k)
+    gate = synthetic.weights(f, k, 0.02, seed=3).cuda()
+    up = synthetic.weights(f, k, 0.05, seed=4).cuda()
+    fw = nv.quantize_weight([gate, up])
+    aq = nv.quantize_act(a.cuda())
+    c1 = nv.gemm(aq, fw)                                              # m x 2f BF16
+    calib, _ = nv.silu_mul_quantize(c1[:, :f], c1[:, f:])              # a calibration run for h's scale
+    h_scale = (calib.scale * 1.1).contiguous()
+    ref, _ = nv.silu_mul_quantize(c1[:, :f], c1[:, f:], h_scale=h_scale)
+    got = nv.gemm_swiglu_quantize(aq, fw, h_scale)
+    torch.cuda.synchronize()
+    nv.check_device_status()
+    assert torch.equal(got.q, ref.q)
+    assert torch.equal(got.sf, ref.sf)
