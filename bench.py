@@ -218,6 +218,19 @@ def run_reference(args):
     return 0
 
 
+def aggregate_over_ranks(total_ms: float, flops_per_step: float, steps: int, world: int, device):
+    """Whole-job throughput of N replicas: the slowest rank's device time over
+    the timed steps (max over ranks: one all-reduce), and TFLOPS = every
+    rank's FLOP / that time (weak scaling: each rank runs the full step)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total = float(t.item())
+    return total, world * flops_per_step * steps / (total * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -283,13 +296,8 @@ def run_ours(args):
     step_ms = [e[0].elapsed_time(e[2]) for e in events]
     gemm_ms = [e[1].elapsed_time(e[2]) for e in events]
     quant_ms = [e[0].elapsed_time(e[1]) for e in events]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms, value = aggregate_over_ranks(sum(step_ms), flops, args.steps, world, device)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
     qs = sorted(step_ms)
     pct = {"p10": qs[int(0.1 * (len(qs) - 1))], "p50": statistics.median(qs), "p90": qs[int(0.9 * (len(qs) - 1))]}
 
