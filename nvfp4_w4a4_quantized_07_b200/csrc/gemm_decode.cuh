@@ -49,7 +49,7 @@ static_assert(SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "TMEM budget");
 // buffers, and the accumulator rows that come from those bytes are never read.
 template <int BT>
 struct Cfg {
-    static constexpr int STAGES = BT >= 64 ? 3 : 4;
+    static constexpr int STAGES = BT >= 64 ? 3 : (BT >= 32 ? 4 : 5);
     static constexpr int A_STAGE = BT * BK_BYTES;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
