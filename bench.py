@@ -50,6 +50,8 @@ def parse():
                     help="small run for ncu: warm-up + K steps only, no sweeps, no e2e")
     ap.add_argument("--probe-peaks", action="store_true",
                     help="measure the dense FP4 tensor-core rate and the HBM read rate with the probe kernels")
+    ap.add_argument("--glue-case", action="store_true",
+                    help="time the MLP glue (silu-mul + dynamic-scale quantisation) on 8192 x 17408, for ncu")
     ap.add_argument("--fused", action="store_true",
                     help="with --decode-case: time nvfp4_linear_decode (quantisation fused in)")
     ap.add_argument("--decode-case", default=None,
@@ -352,17 +354,40 @@ def run_ours(args):
 def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, nv, synthetic, peaks):
     import torch
     out = {}
-    # ---- end to end through the public API: pinned host A in, host C out
+    # ---- end to end through the public API: pinned host A in, host C out.  The
+    # batch is cut into row chunks so that copying chunk j + 1 in, computing
+    # chunk j and copying chunk j - 1 out overlap (PCIe is full duplex); the
+    # static scale makes the chunks independent.
     a_host = p.a.pin_memory()
     c_host = torch.empty((p.m, p.n), dtype=torch.bfloat16).pin_memory()
     a_buf = torch.empty_like(a_dev)
-    aq = nv.quantize_act(a_dev, act_scale=act_scale)
+    chunks = 4 if p.m % 4 == 0 else 1
+    rows = p.m // chunks
+    sl = [slice(j * rows, (j + 1) * rows) for j in range(chunks)]
+    aq_c = [nv.quantize_act(a_dev[sl[j]], act_scale=act_scale) for j in range(chunks)]
+    s_in = torch.cuda.Stream(device)
+    s_out = torch.cuda.Stream(device)
 
     def e2e_step():
-        a_buf.copy_(a_host, non_blocking=True)
-        nv.quantize_act(a_buf, act_scale=act_scale, out=aq)
-        nv.gemm(aq, fw, out=c)
-        c_host.copy_(c, non_blocking=True)
+        s_in.wait_stream(stream)                # a_buf is free once the last step's GEMMs ran
+        ev_in = []
+        with torch.cuda.stream(s_in):
+            for j in range(chunks):
+                a_buf[sl[j]].copy_(a_host[sl[j]], non_blocking=True)
+                ev_in.append(torch.cuda.Event())
+                ev_in[-1].record(s_in)
+        stream.wait_stream(s_out)               # c is free once the last step's copies left
+        ev_c = []
+        for j in range(chunks):
+            stream.wait_event(ev_in[j])
+            nv.quantize_act(a_buf[sl[j]], act_scale=act_scale, out=aq_c[j])
+            nv.gemm(aq_c[j], fw, out=c[sl[j]])
+            ev_c.append(torch.cuda.Event())
+            ev_c[-1].record(stream)
+        with torch.cuda.stream(s_out):
+            for j in range(chunks):
+                s_out.wait_event(ev_c[j])
+                c_host[sl[j]].copy_(c[sl[j]], non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -374,12 +399,16 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
     t0.record(stream)
     for _ in range(n_e2e):
         e2e_step()
+    stream.wait_stream(s_out)
     t1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = t0.elapsed_time(t1) / n_e2e
+    ok = torch.equal(c_host[:4], c[:4].cpu())
     out["e2e"] = {"value": 2.0 * p.m * p.n * p.k / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                   "h2d_bytes_per_step": a_host.numel() * a_host.element_size(),
-                  "d2h_bytes_per_step": c_host.numel() * c_host.element_size(), "ms_per_step": e2e_ms}
+                  "d2h_bytes_per_step": c_host.numel() * c_host.element_size(), "ms_per_step": e2e_ms,
+                  "pipeline": f"{chunks} row chunks: copy in / compute / copy out overlapped on 3 streams",
+                  "host_result_matches_device": bool(ok)}
 
     # ---- dynamic activation scale (amax pass + quantise) for reference
     ws = nv.quant_workspace(device)
@@ -617,6 +646,44 @@ def run_probe_peaks(args):
     return 0
 
 
+def run_glue_case(args):
+    """The MLP glue alone: h = bf16(silu(g) * u) with a dynamic scale and the
+    stored h, quantised; 8192 x 17408 (L2 flushed before each launch)."""
+    import torch
+
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+
+    nvbuild.build()
+    nv.load()
+    device = torch.device("cuda", 0)
+    m, f = 8192, synthetic.MLP_INTERMEDIATE
+    gu = synthetic.mlp_glue_inputs(m, f).to(device)
+    g, u = gu[:, :f], gu[:, f:]
+    ws = nv.quant_workspace(device)
+    h = torch.empty((m, f), dtype=torch.bfloat16, device=device)
+    out = nv.silu_mul_quantize(g, u, workspace=ws, h_out=h)[0]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    times = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        torch.cuda._sleep(400_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        nv.silu_mul_quantize(g, u, workspace=ws, out=out, h_out=h)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    nbytes = m * f * (2 * 2 + 2 + 2 + 0.5 + 1 / 16)
+    print(json.dumps({"glue_case": f"{m}x{f}", "ms": ms, "GB/s": nbytes / (ms * 1e-3) / 1e9, "steps": args.steps}),
+          flush=True)
+    return 0
+
+
 def run_decode_case(args):
     """One decode-shaped GEMM (``m<M>_<shape>``), L2 flushed before each launch."""
     import torch
@@ -666,6 +733,8 @@ def main():
         return run_decode_case(args)
     if args.probe_peaks:
         return run_probe_peaks(args)
+    if args.glue_case:
+        return run_glue_case(args)
     return run_ours(args)
 
 
