@@ -412,6 +412,7 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
 
     # ---- dynamic activation scale (amax pass + quantise) for reference
     ws = nv.quant_workspace(device)
+    aq = nv.quantize_act(a_dev, act_scale=act_scale)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     for _ in range(3):
         nv.quantize_act(a_dev, workspace=ws, out=aq)
