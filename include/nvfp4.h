@@ -56,7 +56,7 @@ extern "C" {
 typedef enum {
     NVFP4_OK = 0,
     NVFP4_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad segment table, ... */
-    NVFP4_ERR_UNSUPPORTED = 2, /* a shape or mode this build does not handle */
+    NVFP4_ERR_UNSUPPORTED = 2, /* a shape or mode this library does not handle */
     NVFP4_ERR_ALIGNMENT = 3,   /* a pointer or leading dimension is not 16-byte aligned */
     NVFP4_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
     NVFP4_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out */

@@ -103,7 +103,7 @@ nvfp4_status device_state(DeviceState** out)
 }
 
 // ---------------------------------------------------------------------------
-// TMA descriptors through the driver entry point (no link-time libcuda).
+// TMA descriptors through the CUDA driver API entry point (no link-time libcuda).
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;

@@ -1,7 +1,7 @@
 """Shared helpers for the GPU parity tests: marshalling between the oracle's
-numpy view and the library's device buffers, and the tolerance check that
-north-stars the GEMM parity (per element 1e-3 * |A_hat row| * |W_hat row|,
-relative Frobenius 2e-3, both before the BF16 cast)."""
+numpy view and the library's device buffers, and the tolerance check of the
+GEMM parity (per element 1e-3 * |A_hat row| * |W_hat row|, relative Frobenius
+2e-3, both before the BF16 cast)."""
 from __future__ import annotations
 
 import numpy as np
