@@ -66,6 +66,7 @@ def lib():
         L.oracle_gemm.argtypes = [P, P, I, I, I, P]
         L.oracle_bf16_round.argtypes = [P, I, P]
         L.oracle_silu_mul_bf16.argtypes = [P, P, I, P]
+        L.oracle_gdn_gates.argtypes = [P, P, I, I, I, P, P, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -244,6 +245,22 @@ def silu_mul_bf16(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
     out = np.empty(g_bits.size, np.uint16)
     lib().oracle_silu_mul_bf16(_ptr(g_bits), _ptr(u_bits), g_bits.size, _ptr(out))
     return out
+
+
+def gdn_gates(a, b, A_log, dt_bias):
+    """GDN gates in FP64: ``g = -exp(A_log) * softplus(a + dt_bias)`` and
+    ``beta = sigmoid(b)`` for m x heads inputs ``a``, ``b`` (FP32 views)."""
+    a = _f32(a)
+    b = _f32(b)
+    m, heads = a.shape
+    if b.shape != (m, heads):
+        raise ValueError("a and b must have the same shape")
+    A_log = _f32(A_log).ravel()
+    dt_bias = _f32(dt_bias).ravel()
+    g = np.empty((m, heads), np.float64)
+    beta = np.empty((m, heads), np.float64)
+    lib().oracle_gdn_gates(_ptr(a), _ptr(b), m, heads, heads, _ptr(A_log), _ptr(dt_bias), _ptr(g), _ptr(beta))
+    return g, beta
 
 
 def num_threads() -> int:

@@ -285,6 +285,31 @@ void oracle_silu_mul_bf16(const uint16_t* g, const uint16_t* u, int64_t n, uint1
     }
 }
 
+/* -------------------------------------------------------------------------
+ * Gated DeltaNet gates from the two head-wide segments a and b of the fused
+ * input projection ("Why Gated DeltaNet Survives 4-Bit Quantization", page
+ * summary, "Gated DeltaNet Mechanics"): the forget gate in log space
+ *     g = -exp(A_log[h]) * softplus(a + dt_bias[h]),  softplus(x) = log(1 + e^x),
+ * and the correction scale beta = sigmoid(b) = 1 / (1 + e^-b) (the pages name
+ * beta_t but its formula is lost in the extracted text; the sigmoid of the b
+ * projection is the reading taken).  FP64 throughout.
+ * ------------------------------------------------------------------------- */
+static double softplus64(double x)
+{
+    /* log(1 + e^x) without overflow: max(x, 0) + log1p(e^-|x|) */
+    return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)));
+}
+
+void oracle_gdn_gates(const float* a, const float* b, int64_t m, int64_t heads, int64_t ld,
+                      const float* A_log, const float* dt_bias, double* g, double* beta)
+{
+    for (int64_t r = 0; r < m; ++r)
+        for (int64_t h = 0; h < heads; ++h) {
+            g[r * heads + h] = -exp((double)A_log[h]) * softplus64((double)a[r * ld + h] + (double)dt_bias[h]);
+            beta[r * heads + h] = 1.0 / (1.0 + exp(-(double)b[r * ld + h]));
+        }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

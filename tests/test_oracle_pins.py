@@ -406,3 +406,58 @@ def test_synthetic_inputs_are_seeded_and_shaped():
     assert (a1[:, c1].float().abs().mean() > 30).item()
     p = synthetic.gdn_in_proj(m=8, k=64)
     assert p.n == 12384 and p.widths == [2048, 2048, 4096, 4096, 48, 48]
+
+
+def test_gdn_gates_closed_forms(oracle_lib):
+    """The Gated DeltaNet gates ("Why Gated DeltaNet Survives 4-Bit
+    Quantization", page summary, "Gated DeltaNet Mechanics"; abstract,
+    mechanism (ii) for the sigmoid) at points with known values."""
+    ln3 = float(np.float32(np.log(3.0)))
+    lnem1 = float(np.float32(np.log(np.e - 1.0)))          # softplus(ln(e - 1)) = 1
+    a = np.array([[0.0, 0.0, lnem1, 1.0, 60.0, -60.0]], np.float32)
+    b = np.array([[0.0, ln3, -ln3, 30.0, -30.0, 1.0]], np.float32)
+    A_log = np.array([0.0, ln3, 0.0, 0.0, 0.0, 0.0], np.float32)
+    dt_bias = np.array([0.0, 0.0, 0.0, -1.0, 0.0, 0.0], np.float32)
+    g, beta = oracle.gdn_gates(a, b, A_log, dt_bias)
+    e3 = np.exp(np.float64(ln3))
+    np.testing.assert_allclose(g[0, 0], -np.log(2.0), rtol=1e-15)
+    np.testing.assert_allclose(g[0, 1], -e3 * np.log(2.0), rtol=1e-15)      # the per-head decay rate scales
+    np.testing.assert_allclose(g[0, 2], -np.log1p(np.exp(np.float64(lnem1))), rtol=1e-15)
+    assert abs(g[0, 2] + 1.0) < 1e-7
+    np.testing.assert_allclose(g[0, 3], -np.log(2.0), rtol=1e-15)           # dt_bias shifts the argument
+    np.testing.assert_allclose(g[0, 4], -60.0, rtol=1e-15)                  # softplus(x) -> x
+    np.testing.assert_allclose(g[0, 5], -np.exp(-60.0), rtol=1e-12)         # softplus(x) -> e^x
+    np.testing.assert_allclose(beta[0, :3], [0.5, 0.75, 0.25], rtol=1e-7)
+    np.testing.assert_allclose(beta[0, 3], 1.0 - np.exp(-30.0), rtol=1e-15)
+    np.testing.assert_allclose(beta[0, 4], np.exp(-30.0), rtol=1e-12)
+    assert np.all(g < 0) and np.all((beta > 0) & (beta < 1))
+
+
+def test_gdn_gates_identities(oracle_lib):
+    """softplus(x) - softplus(-x) = x, sigmoid(x) + sigmoid(-x) = 1 and
+    softplus' = sigmoid: the g and beta paths checked against each other, per
+    head, on random values."""
+    rng = np.random.default_rng(21)
+    m, heads = 64, 48
+    x = rng.normal(0, 6, (m, heads)).astype(np.float32)
+    A_log = rng.normal(0, 1, heads).astype(np.float32)
+    zero = np.zeros(heads, np.float32)
+    g_p, s_p = oracle.gdn_gates(x, x, A_log, zero)
+    g_n, s_n = oracle.gdn_gates(-x, -x, A_log, zero)
+    rate = np.exp(A_log.astype(np.float64))
+    np.testing.assert_allclose((g_n - g_p) / rate, x.astype(np.float64), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s_p + s_n, 1.0, rtol=1e-15)
+    # dt_bias enters as a shift of a: g(a, dt) = g(a + dt, 0)
+    dt = rng.normal(0, 1, heads).astype(np.float32)
+    y = (x.astype(np.float64) + dt).astype(np.float32)
+    exact = (x.astype(np.float64) + dt) == y.astype(np.float64)
+    g_dt, _ = oracle.gdn_gates(x, x, A_log, dt)
+    g_y, _ = oracle.gdn_gates(y, y, A_log, zero)
+    np.testing.assert_array_equal(g_dt[exact], g_y[exact])
+    # central difference of -g / rate (softplus) equals beta (sigmoid)
+    h = np.float32(2.0 ** -8)
+    lo, hi = (x - h).astype(np.float32), (x + h).astype(np.float32)
+    g_lo, _ = oracle.gdn_gates(lo, lo, np.zeros(heads, np.float32), zero)
+    g_hi, _ = oracle.gdn_gates(hi, hi, np.zeros(heads, np.float32), zero)
+    deriv = -(g_hi - g_lo) / (hi.astype(np.float64) - lo.astype(np.float64))
+    np.testing.assert_allclose(deriv, s_p, atol=2e-6)
