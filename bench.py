@@ -427,6 +427,20 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
     out["dynamic_act_scale"] = {"value": 2.0 * p.m * p.n * p.k / (dyn_ms * 1e-3) / 1e12, "unit": UNIT,
                                 "ms_per_step": dyn_ms}
 
+    # ---- the same GEMM with the Gated DeltaNet gates computed in its epilogue
+    # from the last two (head-wide) segments, against the plain GEMM
+    if len(p.widths) >= 2 and p.widths[-1] == p.widths[-2]:
+        heads = p.widths[-1]
+        A_log, dt_bias = (t.to(device) for t in synthetic.gdn_gate_params(heads))
+        g = torch.empty((p.m, heads), dtype=torch.float32, device=device)
+        beta = torch.empty_like(g)
+        a_col = p.n - 2 * heads
+        ms_plain = _timed(lambda: nv.gemm(aq, fw, out=c), flush, stream, device)
+        ms_gdn = _timed(lambda: nv.gemm_gdn(aq, fw, a_col, a_col + heads, A_log, dt_bias, out=c, g=g, beta=beta),
+                        flush, stream, device)
+        out["gdn_gate_epilogue"] = {"heads": heads, "gemm_ms": ms_plain, "gemm_gdn_ms": ms_gdn,
+                                    "overhead_pct": 100.0 * (ms_gdn / ms_plain - 1.0)}
+
     # ---- decode sweep: HBM GB/s of the small-M GEMM (L2 flushed before each launch)
     if not args.no_decode:
         dec = {}

@@ -190,6 +190,48 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * nvfp4_gemm_gdn - nvfp4_gemm (BF16 output) whose epilogue also computes the
+ * Gated DeltaNet gates from two head-wide column ranges of the fused input
+ * projection ("Why Gated DeltaNet Survives 4-Bit Quantization", page summary,
+ * "Gated DeltaNet Mechanics": the log-space forget gate; abstract, mechanism
+ * (ii): the sigmoid parameterization, read as beta = sigmoid(b)).  With
+ * x = the stored BF16 value C[i, j] (FP32 arithmetic from there):
+ *
+ *   g[i, h]    = -exp(A_log[h]) * softplus(C[i, a_col + h] + dt_bias[h])
+ *   beta[i, h] = 1 / (1 + exp(-C[i, b_col + h]))
+ *
+ * C is written exactly as nvfp4_gemm writes it for the same arguments; the
+ * gates are computed by the CTA that produces those columns, from the values
+ * it stores, so they cost no second pass over C.
+ *
+ *   gates->a_col, b_col  first output column of the a and b ranges; each
+ *                        range [col, col + heads) lies within [0, n).
+ *   gates->heads         number of value heads, >= 1.
+ *   gates->A_log,
+ *   gates->dt_bias       device FP32 [heads] (the layer's parameters).
+ *   gates->g, beta       device FP32 outputs, m rows of heads values, row
+ *                        stride ldg >= heads elements.
+ * Other arguments and errors as nvfp4_gemm; odt must be NVFP4_OUT_BF16
+ * (NVFP4_ERR_INVALID_ARG otherwise).
+ * ---------------------------------------------------------------------- */
+typedef struct nvfp4_gdn_gates {
+    int32_t a_col;
+    int32_t b_col;
+    int32_t heads;
+    const float* A_log;
+    const float* dt_bias;
+    float* g;
+    float* beta;
+    int64_t ldg;
+} nvfp4_gdn_gates;
+
+NVFP4_API nvfp4_status nvfp4_gemm_gdn(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
+                                      const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t n, int64_t k,
+                                      const nvfp4_segment* segs, int nsegs, void* c, int64_t ldc,
+                                      const nvfp4_gdn_gates* gates, void* workspace, size_t ws_bytes,
+                                      uint32_t flags, void* stream);
+
+/* ------------------------------------------------------------------------
  * nvfp4_gemm_swiglu_quantize - the gate/up GEMM of a gated MLP with its glue
  * fused into the epilogue: for the fused weight [gate (f rows); up (f rows)]
  * (2f x k, e.g. two separately calibrated modules with their own segment

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: 
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
             "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
-            "nvfp4_linear_decode", "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc",
+            "nvfp4_linear_decode", "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc", "nvfp4_gemm_gdn",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
 NVFP4_NOALLOC_MAX_M = 16
@@ -42,6 +42,12 @@ class NVFP4Error(RuntimeError):
 
 class Segment(ctypes.Structure):
     _fields_ = [("col_begin", ctypes.c_int64), ("col_end", ctypes.c_int64), ("w_global_scale", ctypes.c_float)]
+
+
+class GdnGates(ctypes.Structure):
+    _fields_ = [("a_col", ctypes.c_int32), ("b_col", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("g", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("ldg", ctypes.c_int64)]
 
 
 _lib = None
@@ -72,6 +78,9 @@ def load():
     L.nvfp4_silu_mul_quantize.restype = INT
     L.nvfp4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64, P, SZ, U32, P]
     L.nvfp4_gemm.restype = INT
+    L.nvfp4_gemm_gdn.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, I64,
+                                 ctypes.POINTER(GdnGates), P, SZ, U32, P]
+    L.nvfp4_gemm_gdn.restype = INT
     L.nvfp4_gemm_swiglu_quantize.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, P, P, P]
     L.nvfp4_gemm_swiglu_quantize.restype = INT
     L.nvfp4_linear_decode.argtypes = [P, INT, I64, I64, I64, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P, INT,
@@ -294,6 +303,43 @@ def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NV
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(segments),
         _ptr(out), odt, out.stride(0), _ptr(workspace), ws_bytes, flags, _stream(out.device)))
     return out
+
+
+def gemm_gdn(a: QuantizedActivation, w: FusedWeight, a_col: int, b_col: int, A_log, dt_bias, flags: int = NVFP4_GEMM_AUTO,
+             out=None, g=None, beta=None, workspace=None):
+    """``nvfp4_gemm_gdn``: the fused GDN input projection (BF16 ``C``) with the
+    Gated DeltaNet gates computed in its epilogue from the head-wide column
+    ranges at ``a_col`` and ``b_col`` (one column per head; ``A_log`` and
+    ``dt_bias`` are FP32 device vectors of the head count).  Returns
+    ``(C, g, beta)``, the gates FP32 m x heads."""
+    import torch
+    _require_cuda(A_log, dt_bias)
+    if a.k != w.k:
+        raise ValueError("K mismatch between activations and weight")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32 or A_log.numel() != dt_bias.numel():
+        raise ValueError("A_log and dt_bias must be FP32 vectors of one length (the head count)")
+    heads = A_log.numel()
+    dev = a.q.device
+    if out is None:
+        out = torch.empty((a.m, w.n), dtype=torch.bfloat16, device=dev)
+    if g is None:
+        g = torch.empty((a.m, heads), dtype=torch.float32, device=dev)
+    if beta is None:
+        beta = torch.empty((a.m, heads), dtype=torch.float32, device=dev)
+    if g.stride(0) != beta.stride(0) or g.stride(-1) != 1 or beta.stride(-1) != 1:
+        raise ValueError("g and beta must share a row stride with contiguous rows")
+    A_log, dt_bias = A_log.contiguous(), dt_bias.contiguous()
+    gates = GdnGates(a_col, b_col, heads, A_log.data_ptr(), dt_bias.data_ptr(), g.data_ptr(), beta.data_ptr(),
+                     g.stride(0))
+    arr = segment_array(w.segments)
+    L = load()
+    if workspace is None:
+        workspace = gemm_workspace(a.m, w.n, w.k, flags, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("nvfp4_gemm_gdn", L.nvfp4_gemm_gdn(
+        _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(w.segments),
+        _ptr(out), out.stride(0), ctypes.byref(gates), _ptr(workspace), ws_bytes, flags, _stream(dev)))
+    return out, g, beta
 
 
 def gemm_decode_noalloc(a: QuantizedActivation, w: FusedWeight, out, segments=None):

@@ -72,6 +72,18 @@ struct GemmParams {
     const float* h_scale;
     uint8_t* h_q;
     uint8_t* h_sf;
+    // Gated DeltaNet gates from two head-wide column ranges of the BF16
+    // output (gdn_heads == 0: none): g from columns [gdn_a_col, + heads),
+    // beta from [gdn_b_col, + heads); FP32 outputs m x heads, row stride gdn_ld
+    int gdn_heads, gdn_a_col, gdn_b_col;
+    const float* gdn_A_log;
+    const float* gdn_dt_bias;
+    float* gdn_g;
+    float* gdn_beta;
+    int64_t gdn_ld;
+    // large-M kernel: tile i of the persistent schedule is tile (i + tile_shift)
+    // mod the tile count (0 keeps the column-major order)
+    int tile_shift;
 };
 
 __device__ __forceinline__ float segment_scale(const SegTable& t, int col)
@@ -105,6 +117,90 @@ __device__ __forceinline__ void store8(void* c, int64_t ldc, int out_fp32, int r
         w.z = pack_bf16x2(v[4], v[5]);
         w.w = pack_bf16x2(v[6], v[7]);
         *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(c) + (int64_t)row * ldc + col) = w;
+    }
+}
+
+// The Gated DeltaNet gates ("Why Gated DeltaNet Survives 4-Bit Quantization",
+// page summary, "Gated DeltaNet Mechanics"; the sigmoid for beta from the
+// abstract's mechanism (ii)) from one stored output element x = C[row, col],
+// the BF16 value the next layer would read:
+//   column a_col + h:  g[row, h]    = -exp(A_log[h]) * softplus(x + dt_bias[h])
+//   column b_col + h:  beta[row, h] = 1 / (1 + exp(-x))
+// Both are evaluated so that no intermediate overflows or goes subnormal on
+// the common path (large |x| would otherwise send exp, log1p and the divide
+// into their special-value paths): softplus(t) = max(t, 0) + log1p(exp(-|t|)),
+// which equals t (t >= 17) or exp(t) (t <= -17) to within 2^-25 relative in
+// FP32; the sigmoid as r or e * r with e = exp(-|x|) <= 1 and r the correctly
+// rounded reciprocal of 1 + e, a value in [1, 2].
+__device__ __forceinline__ float gdn_g(float x, float dt_bias, float rate)
+{
+    const float t = __fadd_rn(x, dt_bias);
+    const float at = fabsf(t);
+    const float e = expf(-at);                                   // = exp(t) when t < 0
+    const float tail = t > 0.0f ? t : e;
+    const float sp = at >= 17.0f ? tail : __fadd_rn(fmaxf(t, 0.0f), log1pf(e));
+    return -__fmul_rn(rate, sp);
+}
+
+__device__ __forceinline__ float gdn_beta(float x)
+{
+    const float e = expf(-fabsf(x));
+    const float r = __frcp_rn(__fadd_rn(1.0f, e));
+    return x >= 0.0f ? r : __fmul_rn(e, r);
+}
+
+// Whether output columns [col0, col0 + ncols) hold any gate input.
+__device__ __forceinline__ bool gdn_touches(const GemmParams& p, int col0, int ncols)
+{
+    return p.gdn_heads > 0 && ((col0 < p.gdn_a_col + p.gdn_heads && p.gdn_a_col < col0 + ncols) ||
+                               (col0 < p.gdn_b_col + p.gdn_heads && p.gdn_b_col < col0 + ncols));
+}
+
+// Gates from 4 consecutive stored columns of one row (the decode kernel's
+// output unit); called only where gdn_touches holds.
+__device__ __forceinline__ void gdn_gate4(const GemmParams& p, int row, int col, float x0, float x1, float x2, float x3)
+{
+    const float x[4] = {x0, x1, x2, x3};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const unsigned ha = (unsigned)(col + e - p.gdn_a_col), hb = (unsigned)(col + e - p.gdn_b_col);
+        if (ha < (unsigned)p.gdn_heads)
+            p.gdn_g[(int64_t)row * p.gdn_ld + ha] = gdn_g(x[e], p.gdn_dt_bias[ha], expf(p.gdn_A_log[ha]));
+        if (hb < (unsigned)p.gdn_heads) p.gdn_beta[(int64_t)row * p.gdn_ld + hb] = gdn_beta(x[e]);
+    }
+}
+
+// Gates from one 16-row x 32-column BF16 output chunk staged in shared memory
+// (64-byte rows; 16-byte unit u of row r at (u ^ ((r / 2) % 4)) * 16): lane =
+// column; the head's parameters are read once and four rows at a time are
+// unrolled so that their exp/log1p chains overlap (rows are otherwise a
+// serial chain of dependent transcendental steps in a single warp).
+__device__ __forceinline__ void gdn_chunk(const GemmParams& p, const uint8_t* cbuf, int row0, int col0, int lane)
+{
+    const int col = col0 + lane;
+    const unsigned ha = (unsigned)(col - p.gdn_a_col), hb = (unsigned)(col - p.gdn_b_col);
+    const bool is_a = ha < (unsigned)p.gdn_heads, is_b = hb < (unsigned)p.gdn_heads;
+    if (!is_a && !is_b) return;
+    const float dt_bias = is_a ? p.gdn_dt_bias[ha] : 0.0f;
+    const float rate = is_a ? expf(p.gdn_A_log[ha]) : 0.0f;
+    const int rows = min(16, p.m - row0);
+    float* g = p.gdn_g + (int64_t)row0 * p.gdn_ld + ha;
+    float* beta = p.gdn_beta + (int64_t)row0 * p.gdn_ld + hb;
+#pragma unroll 4
+    for (int r = 0; r < 16; ++r) {
+        // every row of the buffer is read (rows past m hold stale values whose
+        // results are dropped), so only the stores are conditional and the
+        // unrolled rows' chains can interleave
+        const uint8_t* src = cbuf + r * 64 + ((((lane >> 3) ^ ((r >> 1) & 3)) << 4) | ((lane & 7) << 1));
+        const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(src));
+        if (is_a) {
+            const float v = gdn_g(x, dt_bias, rate);
+            if (r < rows) g[r * p.gdn_ld] = v;
+        }
+        if (is_b) {
+            const float v = gdn_beta(x);
+            if (r < rows) beta[r * p.gdn_ld] = v;
+        }
     }
 }
 

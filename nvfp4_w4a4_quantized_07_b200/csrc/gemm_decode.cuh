@@ -95,9 +95,13 @@ __device__ __forceinline__ void store4_scaled(const GemmParams& p, int row, int 
     const float o2 = __fmul_rn(v.z, alpha), o3 = __fmul_rn(v.w, alpha);
     if (p.out_fp32)
         *reinterpret_cast<float4*>(static_cast<float*>(p.c) + (int64_t)row * p.ldc + col) = make_float4(o0, o1, o2, o3);
-    else
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col) =
-            make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+    else {
+        const uint2 w = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col) = w;
+        if (gdn_touches(p, col, 4))
+            gdn_gate4(p, row, col, __bfloat162float(__float2bfloat16_rn(o0)), __bfloat162float(__float2bfloat16_rn(o1)),
+                      __bfloat162float(__float2bfloat16_rn(o2)), __bfloat162float(__float2bfloat16_rn(o3)));
+    }
 }
 
 // FQ: the activation quantisation is fused in.  Warps 2 and 3 then quantise

@@ -108,6 +108,44 @@ __device__ __forceinline__ void drain_bf16_plan(int b, int half, uint32_t taddr,
     }
 }
 
+// Gated DeltaNet gates of the warp's 32 x 128 slice, after its stores: the
+// chunks holding gate columns go through the staging buffer once more (j
+// picked at run time; each switch arm indexes `packed` with constants, so it
+// stays in registers) and gdn_chunk reads them there.  One copy of the gate
+// code per kernel, outside the unrolled store loop.
+template <int J>
+__device__ __forceinline__ void stage_chunk_row(uint8_t* cbuf, const uint32_t (&packed)[4][16], int r)
+{
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4*>(cbuf + r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) =
+            make_uint4(packed[J][4 * u], packed[J][4 * u + 1], packed[J][4 * u + 2], packed[J][4 * u + 3]);
+}
+
+__device__ __forceinline__ void gdn_pass(const GemmParams& p, uint8_t* cbuf, const uint32_t (&packed)[4][16], int row0,
+                                         int ncol0, int lane)
+{
+    if (lane == 0) bulk_wait_group_read<0>();  // the last TMA store has read the buffer
+    __syncwarp();
+#pragma unroll 1
+    for (int q = 0; q < 8; ++q) {
+        const int j = q >> 1, hr = q & 1;
+        if (!gdn_touches(p, ncol0 + j * 32, 32)) continue;
+        if ((lane >> 4) == hr) {
+            const int r = lane & 15;
+            switch (j) {
+                case 0: stage_chunk_row<0>(cbuf, packed, r); break;
+                case 1: stage_chunk_row<1>(cbuf, packed, r); break;
+                case 2: stage_chunk_row<2>(cbuf, packed, r); break;
+                default: stage_chunk_row<3>(cbuf, packed, r); break;
+            }
+        }
+        __syncwarp();
+        gdn_chunk(p, cbuf, row0 + 16 * hr, ncol0 + j * 32, lane);
+        __syncwarp();
+    }
+}
+
 namespace large {
 constexpr int BM = 128, BN = 256, BK_BYTES = 128;  // BK = 256 FP4 values per stage
 constexpr int STAGES = 4;
@@ -201,7 +239,8 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
+                const int t = tile + p.tile_shift - (tile + p.tile_shift >= num_tiles ? num_tiles : 0);
+                const int mb = t % p.m_tiles, nb = t / p.m_tiles;
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
                         ok = false;
@@ -377,7 +416,8 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         int i = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int b = i & 1;
-            const int mb = tile % p.m_tiles, nb = tile / p.m_tiles;
+            const int t = tile + p.tile_shift - (tile + p.tile_shift >= num_tiles ? num_tiles : 0);
+            const int mb = t % p.m_tiles, nb = t / p.m_tiles;
             if (!mbar_wait(&acc_full[b], (i >> 1) & 1, kStatusTimeoutAccum)) break;
             tc_fence_after();
             const int row = mb * BM + quad * 32 + lane;
@@ -471,6 +511,7 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                         }
                     }
                 }
+                if (gdn_touches(p, ncol0, 128)) gdn_pass(p, cbuf, packed, row0, ncol0, lane);
             } else {
                 for (int jj = 0; jj < 4; ++jj) {
                     const int j = (ov_rot + jj) & 3;
@@ -822,6 +863,7 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
                         }
                     }
                 }
+                if (gdn_touches(p, ncol0, 128)) gdn_pass(p, cbuf, packed, row0, ncol0, lane);
             } else {
                 for (int jj = 0; jj < 4; ++jj) {
                     const int j = (ov_rot + jj) & 3;

@@ -542,10 +542,11 @@ nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_in_dtype dt, int64_t n, 
     return ok();
 }
 
-nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
-                        const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs, int nsegs,
-                        void* c, nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, uint32_t flags,
-                        void* stream)
+// nvfp4_gemm and nvfp4_gemm_gdn: `gates` (checked by the caller) or NULL.
+static nvfp4_status gemm_impl(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
+                              const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs,
+                              int nsegs, void* c, nvfp4_out_dtype odt, int64_t ldc, const nvfp4_gdn_gates* gates,
+                              void* workspace, size_t ws_bytes, uint32_t flags, void* stream)
 {
     if (m < 0 || n <= 0 || k <= 0 || n % 16 != 0 || k % 32 != 0)
         return fail(NVFP4_ERR_INVALID_ARG, "gemm: need m >= 0, n a positive multiple of 16, k a positive multiple of 32 "
@@ -595,6 +596,16 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     p.a_rowblocks = (int)((m + 127) / 128);
     p.w_rowblocks = (int)((n + 127) / 128);
     p.splits = 1;
+    if (gates != nullptr) {
+        p.gdn_heads = gates->heads;
+        p.gdn_a_col = gates->a_col;
+        p.gdn_b_col = gates->b_col;
+        p.gdn_A_log = gates->A_log;
+        p.gdn_dt_bias = gates->dt_bias;
+        p.gdn_g = gates->g;
+        p.gdn_beta = gates->beta;
+        p.gdn_ld = gates->ldg;
+    }
 
     CUtensorMap ta, tw;
     if (!use_decode && flags != NVFP4_GEMM_FORCE_LARGE_PAIR) {
@@ -606,6 +617,17 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
         if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
+        if (gates != nullptr) {
+            // The gate columns' tiles carry the longest epilogue: schedule them
+            // first, on CTAs [extra, ...) which run one tile fewer than CTAs
+            // [0, extra), so that the slower epilogue overlaps later MMAs
+            // instead of ending the kernel (in column-major order they are
+            // the last tiles when the gate ranges close the fused weight).
+            const int64_t extra = tiles % grid;
+            const int64_t first = (int64_t)((gates->a_col < gates->b_col ? gates->a_col : gates->b_col) / large::BN) *
+                                  p.m_tiles;
+            p.tile_shift = (int)(((first - extra) % tiles + tiles) % tiles);
+        }
         gemm_large_kernel<false><<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tc, p);
         NVFP4_CUDA_TRY(cudaGetLastError());
         return ok();
@@ -655,6 +677,39 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* ac
     else st = launch_decode<64, false>(ta, tw, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
+                        const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs, int nsegs,
+                        void* c, nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, uint32_t flags,
+                        void* stream)
+{
+    return gemm_impl(a_q, a_sf, act_scale_dev, w_q, w_sf, m, n, k, segs, nsegs, c, odt, ldc, nullptr, workspace,
+                     ws_bytes, flags, stream);
+}
+
+nvfp4_status nvfp4_gemm_gdn(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev, const uint8_t* w_q,
+                            const uint8_t* w_sf, int64_t m, int64_t n, int64_t k, const nvfp4_segment* segs,
+                            int nsegs, void* c, int64_t ldc, const nvfp4_gdn_gates* gates, void* workspace,
+                            size_t ws_bytes, uint32_t flags, void* stream)
+{
+    if (gates == nullptr) return fail(NVFP4_ERR_INVALID_ARG, "gemm_gdn: NULL gates");
+    const int64_t heads = gates->heads;
+    if (heads < 1 || gates->a_col < 0 || gates->b_col < 0 || gates->a_col + heads > n || gates->b_col + heads > n)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm_gdn: gate columns [%d, +%d) and [%d, +%d) must lie in [0, n=%lld)",
+                    gates->a_col, gates->heads, gates->b_col, gates->heads, (long long)n);
+    if (gates->ldg < heads)
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm_gdn: ldg %lld < heads %d", (long long)gates->ldg, gates->heads);
+    if (m > 0 && (gates->A_log == nullptr || gates->dt_bias == nullptr || gates->g == nullptr ||
+                  gates->beta == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "gemm_gdn: NULL gate pointer");
+    if (reinterpret_cast<uintptr_t>(gates->A_log) % 4 || reinterpret_cast<uintptr_t>(gates->dt_bias) % 4 ||
+        reinterpret_cast<uintptr_t>(gates->g) % 4 || reinterpret_cast<uintptr_t>(gates->beta) % 4)
+        return fail(NVFP4_ERR_ALIGNMENT, "gemm_gdn: gate vectors must be 4-byte aligned");
+    if (m > 0 && m * gates->ldg >= (1ll << 40))
+        return fail(NVFP4_ERR_UNSUPPORTED, "gemm_gdn: gate outputs too large");
+    return gemm_impl(a_q, a_sf, act_scale_dev, w_q, w_sf, m, n, k, segs, nsegs, c, NVFP4_OUT_BF16, ldc, gates,
+                     workspace, ws_bytes, flags, stream);
 }
 
 nvfp4_status nvfp4_gemm_swiglu_quantize(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,

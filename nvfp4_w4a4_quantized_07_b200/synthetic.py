@@ -21,6 +21,8 @@ from __future__ import annotations
 
 from dataclasses import dataclass, field
 
+import math
+
 import torch
 
 HIDDEN = 5120
@@ -117,6 +119,19 @@ def mlp_gate_up(m: int = 32768, k: int = HIDDEN, inter: int = MLP_INTERMEDIATE) 
 
 def mlp_down_weight(k: int = MLP_INTERMEDIATE, n: int = HIDDEN) -> torch.Tensor:
     return weights(n, k, 0.02, seed=3)
+
+
+def gdn_gate_params(heads: int = 48, seed: int = 9):
+    """Per-head parameters of a Gated DeltaNet layer's gates, drawn the usual
+    way such layers are initialised: ``A_log = log(U(1, 16))`` and ``dt_bias``
+    the inverse softplus of a step size log-uniform in [1e-3, 1e-1].  FP32."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    A_log = torch.log(1.0 + 15.0 * torch.rand(heads, generator=g, dtype=torch.float64))
+    dt = torch.exp(math.log(1e-3) + (math.log(1e-1) - math.log(1e-3)) * torch.rand(heads, generator=g,
+                                                                                    dtype=torch.float64))
+    dt_bias = dt + torch.log(-torch.expm1(-dt))
+    return A_log.float(), dt_bias.float()
 
 
 def mlp_glue_inputs(m: int, f: int, seed: int = 5, gate_std: float = 2.0) -> torch.Tensor:

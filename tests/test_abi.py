@@ -221,3 +221,24 @@ def test_gemm_swiglu_quantize_argument_errors(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, s2, 2, None, FAKE, FAKE, None) == 1                    # no scale
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, s2, 2, FAKE, MISALIGNED, FAKE, None) == 3
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 128, 64, s2, 2, FAKE, FAKE, FAKE, None) == 0                    # empty
+
+
+def test_gemm_gdn_argument_errors(lib):
+    f = lib.nvfp4_gemm_gdn
+    s = _segs((0, 128, 1.0))
+
+    def call(a_col=64, b_col=96, heads=32, ldg=32, ptrs=(FAKE, FAKE, FAKE, FAKE), m=8, n=128):
+        gates = nv.GdnGates(a_col, b_col, heads, *[None if p is None else p.value for p in ptrs], ldg)
+        segs = s if n == 128 else _segs((0, n, 1.0))
+        return f(FAKE, FAKE, FAKE, FAKE, FAKE, m, n, 64, segs, 1, FAKE, n, ctypes.byref(gates), None, 0, 1, None)
+
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 128, 64, s, 1, FAKE, 128, None, None, 0, 1, None) == 1   # no gates
+    assert call(heads=0) == 1
+    assert call(a_col=-1) == 1
+    assert call(a_col=100) == 1                          # a range past n
+    assert call(b_col=97) == 1                           # b range past n
+    assert call(ldg=16) == 1                             # ldg < heads
+    assert call(ptrs=(FAKE, None, FAKE, FAKE)) == 1      # no dt_bias
+    assert call(ptrs=(FAKE, FAKE, FAKE, ctypes.c_void_p(0x10002))) == 3
+    assert call(a_col=100) == 1 and b"gemm_gdn" in lib.nvfp4_get_last_error_string()
+    assert call(m=0) == 0                                # empty
