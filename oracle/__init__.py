@@ -67,6 +67,9 @@ def lib():
         L.oracle_bf16_round.argtypes = [P, I, P]
         L.oracle_silu_mul_bf16.argtypes = [P, P, I, P]
         L.oracle_gdn_gates.argtypes = [P, P, I, I, I, P, P, P, P]
+        L.oracle_fp8_scale_from_amax.argtypes = [ctypes.c_float]
+        L.oracle_fp8_scale_from_amax.restype = ctypes.c_float
+        L.oracle_fp8_quantize.argtypes = [P, I, ctypes.c_float, P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -244,6 +247,19 @@ def silu_mul_bf16(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
     u_bits = np.ascontiguousarray(u_bits, np.uint16).ravel()
     out = np.empty(g_bits.size, np.uint16)
     lib().oracle_silu_mul_bf16(_ptr(g_bits), _ptr(u_bits), g_bits.size, _ptr(out))
+    return out
+
+
+def fp8_scale_from_amax(amax) -> np.float32:
+    """Calibrated per-tensor FP8 KV-cache scale: ``amax / 448`` (1 if 0)."""
+    return np.float32(lib().oracle_fp8_scale_from_amax(float(np.float32(amax))))
+
+
+def fp8_quantize(x, scale) -> np.ndarray:
+    """E4M3 bytes of ``x * (1 / scale)`` (FP32, RNE, saturating), same shape."""
+    x = _f32(x)
+    out = np.empty(x.shape, np.uint8)
+    lib().oracle_fp8_quantize(_ptr(x), x.size, float(np.float32(scale)), _ptr(out))
     return out
 
 

@@ -286,6 +286,35 @@ void oracle_silu_mul_bf16(const uint16_t* g, const uint16_t* u, int64_t n, uint1
 }
 
 /* -------------------------------------------------------------------------
+ * Calibrated FP8 KV cache (abstract: calibrated FP8 KV-cache scales cost no
+ * performance and ship with the recipe; Glonce article, "How to use it";
+ * aiany.app, "Mechanistic notes").  The pages give no formula; the readings:
+ *   - one FP32 scale per tensor (K and V each), calibrated as
+ *     s = amax / 448 (448 = the largest E4M3 value; one FP32 division), or
+ *     s = 1 if that quotient is 0;
+ *   - stored byte = E4M3_rne_satfinite(x * inv_s), inv_s = 1 / s (FP32,
+ *     correctly rounded; FLT_MAX if the reciprocal overflows), the sign bit
+ *     copied from the FP32 product (so -0 and small negatives give 0x80);
+ *   - the value read back is decode(byte) * s.
+ * ------------------------------------------------------------------------- */
+float oracle_fp8_scale_from_amax(float amax)
+{
+    volatile float s = amax / 448.0f;
+    return s == 0.0f ? 1.0f : s;
+}
+
+void oracle_fp8_quantize(const float* x, int64_t n, float scale, uint8_t* out)
+{
+    volatile float inv = 1.0f / scale;
+    if (isinf(inv)) inv = FLT_MAX;
+    for (int64_t i = 0; i < n; ++i) {
+        volatile float y = x[i] * inv;
+        uint8_t c = oracle_e4m3_encode_positive(y);
+        out[i] = signbit(y) ? (uint8_t)(c | 0x80) : c;
+    }
+}
+
+/* -------------------------------------------------------------------------
  * Gated DeltaNet gates from the two head-wide segments a and b of the fused
  * input projection ("Why Gated DeltaNet Survives 4-Bit Quantization", page
  * summary, "Gated DeltaNet Mechanics"): the forget gate in log space

@@ -461,3 +461,63 @@ def test_gdn_gates_identities(oracle_lib):
     g_hi, _ = oracle.gdn_gates(hi, hi, np.zeros(heads, np.float32), zero)
     deriv = -(g_hi - g_lo) / (hi.astype(np.float64) - lo.astype(np.float64))
     np.testing.assert_allclose(deriv, s_p, atol=2e-6)
+
+
+# --------------------------------------------------------------------------- FP8 KV cache
+def _e4m3_value(code: int) -> float:
+    """E4M3 (fn) value of a byte, from the format's definition: bias 7, three
+    mantissa bits, exponent field 0 subnormal, 0x7f/0xff NaN."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e, m = (code >> 3) & 15, code & 7
+    mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return sign * mag
+
+
+def test_fp8_codes_round_trip_and_ties(oracle_lib):
+    """Every finite E4M3 byte survives value -> byte; the midpoint of two
+    neighbouring values rounds to the even mantissa; beyond 448 saturates
+    ("calibrated FP8 KV-cache", abstract; Glonce "How to use it")."""
+    codes = [c for c in range(256) if c & 0x7F != 0x7F]
+    vals = np.array([_e4m3_value(c) for c in codes], np.float32)
+    vals[codes.index(0x80)] = np.float32(-0.0)
+    np.testing.assert_array_equal(oracle.fp8_quantize(vals, 1.0), np.array(codes, np.uint8))
+    pos = [c for c in range(0x7F)]
+    mids = np.array([(_e4m3_value(c) + _e4m3_value(c + 1)) / 2 for c in pos[:-1]], np.float32)
+    got = oracle.fp8_quantize(mids, 1.0)
+    want = np.array([c if c % 2 == 0 else c + 1 for c in pos[:-1]], np.uint8)
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(oracle.fp8_quantize(-mids, 1.0), want | 0x80)
+    big = np.array([448.0, 464.0, 479.9, 480.0, 1e30, np.inf], np.float32)
+    np.testing.assert_array_equal(oracle.fp8_quantize(big, 1.0), np.full(6, 0x7E, np.uint8))
+    np.testing.assert_array_equal(oracle.fp8_quantize(-big, 1.0), np.full(6, 0xFE, np.uint8))
+
+
+def test_fp8_matches_torch_float8_in_range(oracle_lib):
+    """Inside +-448 the bytes equal PyTorch's float8_e4m3fn cast (an independent
+    round-to-nearest-even implementation), subnormals included."""
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal(200_000) * np.exp2(rng.uniform(-14, 8.7, 200_000))).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.fp8_quantize(x, 1.0), want)
+
+
+def test_fp8_scale_is_a_divisor_and_bounds_the_error(oracle_lib):
+    """s = amax / 448 maps the largest magnitude onto 448; values are divided
+    by s (quantize(x, 2s) == quantize(x / 2, s)); read back as byte * s the
+    error is at most half an E4M3 step."""
+    rng = np.random.default_rng(32)
+    x = (rng.standard_normal((256, 512)) * 3.0).astype(np.float32)
+    x[17, 300] = -41.5
+    amax = np.float32(np.abs(x).max())
+    s = oracle.fp8_scale_from_amax(amax)
+    assert s == np.float32(amax / np.float32(448.0))
+    assert oracle.fp8_scale_from_amax(0.0) == 1.0 and oracle.fp8_scale_from_amax(448.0) == 1.0
+    q = oracle.fp8_quantize(x, s)
+    assert q[17, 300] == 0xFE
+    np.testing.assert_array_equal(oracle.fp8_quantize(x, np.float32(2.0) * s), oracle.fp8_quantize(x / 2, s))
+    back = np.vectorize(_e4m3_value)(q.astype(np.int64)) * np.float64(s)
+    err = np.abs(back - x.astype(np.float64))
+    bound = 2.0 ** -4 * np.abs(x) * (1 + 2.0 ** -20) + 2.0 ** -10 * np.float64(s)
+    assert np.all(err <= bound)
+    assert np.all(np.sign(back[np.abs(back) > 0]) == np.sign(x[np.abs(back) > 0]))
