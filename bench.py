@@ -441,6 +441,25 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
         out["gdn_gate_epilogue"] = {"heads": heads, "gemm_ms": ms_plain, "gemm_gdn_ms": ms_gdn,
                                     "overhead_pct": 100.0 * (ms_gdn / ms_plain - 1.0)}
 
+    # ---- calibrated FP8 KV cache: one layer's new K/V rows quantised and
+    # scattered into shuffled cache slots (prefill and decode sizes)
+    kv = {}
+    for tokens in (8192, 16):
+        k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens))
+        ks = torch.empty(1, dtype=torch.float32, device=device)
+        vs = torch.empty(1, dtype=torch.float32, device=device)
+        nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
+        nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
+        gen = torch.Generator().manual_seed(tokens)
+        slots = torch.randperm(2 * tokens, generator=gen)[:tokens].to(torch.int64).to(device)
+        kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
+        vc = torch.empty_like(kc)
+        ms = _timed(lambda: nv.kv_cache_quantize_fp8(k_rows, v_rows, ks, vs, kc, vc, slots), flush, stream, device)
+        nbytes = 2 * k_rows.numel() * (k_rows.element_size() + 1) + slots.numel() * 8
+        kv[f"tokens{tokens}_width{k_rows.shape[1]}"] = {
+            "us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    out["kv_cache_fp8"] = {"bytes": "K and V in (bf16) + cache bytes out + int64 slot table", "shapes": kv}
+
     # ---- decode sweep: HBM GB/s of the small-M GEMM (L2 flushed before each launch)
     if not args.no_decode:
         dec = {}

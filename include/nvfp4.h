@@ -351,6 +351,58 @@ NVFP4_API nvfp4_status nvfp4_gemm_decode_noalloc(const uint8_t* a_q, const uint8
                                        int64_t ldc, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Calibrated FP8 (E4M3) KV cache.  The recipe pairs the NVFP4 W4A4 layers
+ * with an FP8 KV cache whose per-tensor scales are calibrated offline and
+ * shipped with the checkpoint ("Why Gated DeltaNet Survives 4-Bit
+ * Quantization": abstract; Glonce article, "How to use it"; aiany.app,
+ * "Mechanistic notes").  The pages give no formula; this library reads it as
+ *
+ *   scale s  = amax / 448 over the calibration data (448 = largest E4M3
+ *              value; one FP32 division), s = 1 if that is 0;
+ *   byte     = E4M3 round-to-nearest-even, saturating to +-448, of x * (1/s)
+ *              (1/s correctly rounded in FP32, FLT_MAX if it overflows);
+ *   value    = e4m3(byte) * s when attention reads the cache.
+ * ---------------------------------------------------------------------- */
+
+/* nvfp4_fp8_calibrate - fold one calibration batch into a running amax and
+ * refresh the scale: *amax_inout = max(*amax_inout, max |x|), then
+ * *scale_out = *amax_inout / 448 (1 if 0).  Start *amax_inout at 0.
+ *
+ *   x, dt, rows, width, ld  rows x width BF16/FP32 values (device), row
+ *                           stride ld elements; width a multiple of 16, rows
+ *                           16-byte aligned.  rows may be 0 (scale refresh).
+ *   amax_inout_dev          device float, non-negative (running maximum).
+ *   scale_out_dev           device float, receives the scale.
+ * Errors: NVFP4_ERR_INVALID_ARG (shape, NULL), NVFP4_ERR_ALIGNMENT. */
+NVFP4_API nvfp4_status nvfp4_fp8_calibrate(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t width, int64_t ld,
+                                           float* amax_inout_dev, float* scale_out_dev, void* stream);
+
+/* nvfp4_kv_cache_quantize_fp8 - quantise the K and V rows of `tokens` new
+ * tokens to E4M3 with their calibrated scales and store each token's row in
+ * its cache slot, in one launch.
+ *
+ *   k, v, dt          device, tokens x width BF16/FP32 (width = KV heads x
+ *                     head size, a multiple of 16), row strides ld_k, ld_v
+ *                     elements, rows 16-byte aligned.
+ *   slot_mapping      device int64[tokens]: the cache row of each token; a
+ *                     negative entry (padding) or one >= num_slots is
+ *                     skipped.  NULL: token t goes to slot t (then tokens <=
+ *                     num_slots).
+ *   k_scale_dev,
+ *   v_scale_dev       device floats, the calibrated scales.
+ *   k_cache, v_cache  device, num_slots rows of width bytes, row stride
+ *                     cache_ld bytes (a multiple of 16, >= width); rows not
+ *                     named by the slot table are left untouched.
+ * Requires tokens x width / 16 < 2^31.  Errors: NVFP4_ERR_INVALID_ARG,
+ * NVFP4_ERR_UNSUPPORTED, NVFP4_ERR_ALIGNMENT, NVFP4_ERR_CUDA. */
+NVFP4_API nvfp4_status nvfp4_kv_cache_quantize_fp8(const void* k, const void* v, nvfp4_in_dtype dt, int64_t tokens,
+                                                   int64_t width, int64_t ld_k, int64_t ld_v,
+                                                   const int64_t* slot_mapping, int64_t num_slots,
+                                                   const float* k_scale_dev, const float* v_scale_dev,
+                                                   uint8_t* k_cache, uint8_t* v_cache, int64_t cache_ld,
+                                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * Diagnostics.
  * ---------------------------------------------------------------------- */
 

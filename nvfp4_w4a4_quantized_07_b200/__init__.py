@@ -29,6 +29,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: 
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
             "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
             "nvfp4_linear_decode", "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc", "nvfp4_gemm_gdn",
+            "nvfp4_fp8_calibrate", "nvfp4_kv_cache_quantize_fp8",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
 NVFP4_NOALLOC_MAX_M = 16
@@ -81,6 +82,10 @@ def load():
     L.nvfp4_gemm_gdn.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, I64,
                                  ctypes.POINTER(GdnGates), P, SZ, U32, P]
     L.nvfp4_gemm_gdn.restype = INT
+    L.nvfp4_fp8_calibrate.argtypes = [P, INT, I64, I64, I64, P, P, P]
+    L.nvfp4_fp8_calibrate.restype = INT
+    L.nvfp4_kv_cache_quantize_fp8.argtypes = [P, P, INT, I64, I64, I64, I64, P, I64, P, P, P, P, I64, P]
+    L.nvfp4_kv_cache_quantize_fp8.restype = INT
     L.nvfp4_gemm_swiglu_quantize.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, P, P, P]
     L.nvfp4_gemm_swiglu_quantize.restype = INT
     L.nvfp4_linear_decode.argtypes = [P, INT, I64, I64, I64, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P, INT,
@@ -340,6 +345,48 @@ def gemm_gdn(a: QuantizedActivation, w: FusedWeight, a_col: int, b_col: int, A_l
         _ptr(a.q), _ptr(a.sf), _ptr(a.scale), _ptr(w.q), _ptr(w.sf), a.m, w.n, w.k, arr, len(w.segments),
         _ptr(out), out.stride(0), ctypes.byref(gates), _ptr(workspace), ws_bytes, flags, _stream(dev)))
     return out, g, beta
+
+
+def fp8_calibrate(x, amax, scale):
+    """``nvfp4_fp8_calibrate``: fold ``x`` (BF16/FP32, leading dimension =
+    rows, the rest flattened into the width) into the running ``amax`` and
+    write the calibrated FP8 scale ``amax / 448`` into ``scale`` (both
+    1-element FP32 device tensors; start ``amax`` at 0)."""
+    _require_cuda(x, amax, scale)
+    x2 = x.reshape(x.shape[0], -1) if x.dim() != 2 else x
+    _check("nvfp4_fp8_calibrate", load().nvfp4_fp8_calibrate(
+        _ptr(x2), _in_dtype(x2), x2.shape[0], x2.shape[1], x2.stride(0), _ptr(amax), _ptr(scale),
+        _stream(x.device)))
+    return scale
+
+
+def kv_cache_quantize_fp8(k, v, k_scale, v_scale, k_cache, v_cache, slot_mapping=None):
+    """``nvfp4_kv_cache_quantize_fp8``: quantise the new tokens' K and V
+    (``tokens x ...``, BF16/FP32) to E4M3 with their calibrated scales and
+    store token t's row in cache row ``slot_mapping[t]`` (int64; negative =
+    skip; None = slot t).  The caches are uint8 ``num_slots x ...`` tensors
+    whose rows are written in place."""
+    import torch
+    _require_cuda(k, v, k_scale, v_scale, k_cache, v_cache, slot_mapping)
+    if k.shape != v.shape or k.dtype != v.dtype:
+        raise ValueError("k and v must have one shape and dtype")
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8 or k_cache.shape != v_cache.shape:
+        raise ValueError("the caches must be uint8 tensors of one shape")
+    if k_cache.stride(0) != v_cache.stride(0):
+        raise ValueError("the caches must share a row stride")
+    if slot_mapping is not None and (slot_mapping.dtype != torch.int64 or slot_mapping.numel() != k.shape[0]):
+        raise ValueError("slot_mapping must be int64 with one entry per token")
+    k2 = k.reshape(k.shape[0], -1)
+    v2 = v.reshape(v.shape[0], -1)
+    kc = k_cache.view(k_cache.shape[0], -1)     # a view: the kernel writes the caller's rows
+    vc = v_cache.view(v_cache.shape[0], -1)
+    if kc.shape[1] != k2.shape[1]:
+        raise ValueError("cache rows and K/V rows differ in width")
+    _check("nvfp4_kv_cache_quantize_fp8", load().nvfp4_kv_cache_quantize_fp8(
+        _ptr(k2), _ptr(v2), _in_dtype(k2), k2.shape[0], k2.shape[1], k2.stride(0), v2.stride(0),
+        _ptr(slot_mapping), kc.shape[0], _ptr(k_scale), _ptr(v_scale), _ptr(kc), _ptr(vc), kc.stride(0),
+        _stream(k.device)))
+    return k_cache, v_cache
 
 
 def gemm_decode_noalloc(a: QuantizedActivation, w: FusedWeight, out, segments=None):

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnvfp4.so")
 SOURCES = [os.path.join(CSRC, "nvfp4_lib.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "quant.cuh", "gemm_common.cuh", "gemm_large.cuh",
-                                                 "gemm_decode.cuh")] + [os.path.join(ROOT, "include", "nvfp4.h")]
+                                                 "gemm_decode.cuh", "kv_fp8.cuh")] + [os.path.join(ROOT, "include", "nvfp4.h")]
 PROBES_LIB = os.path.join(PKG, "libnvfp4_probes.so")
 PROBES_SOURCES = [os.path.join(CSRC, "probes.cu")]
 PROBES_DEPS = PROBES_SOURCES + [os.path.join(CSRC, "ptx.cuh")]

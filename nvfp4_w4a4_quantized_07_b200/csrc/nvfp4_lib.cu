@@ -17,6 +17,7 @@
 #include "../../include/nvfp4.h"
 #include "gemm_decode.cuh"
 #include "gemm_large.cuh"
+#include "kv_fp8.cuh"
 #include "quant.cuh"
 
 using namespace nvfp4;
@@ -169,19 +170,25 @@ nvfp4_status check_quant_input(const void* x, nvfp4_in_dtype dt, int64_t rows, i
     return NVFP4_OK;
 }
 
-nvfp4_status launch_amax(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t k, int64_t ld, void* ws,
-                         cudaStream_t s, int sms)
+// max(*out, amax(x)) into *out (float bits; *out holds a non-negative float).
+nvfp4_status launch_amax_into(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t k, int64_t ld, unsigned int* out,
+                              cudaStream_t s, int sms)
 {
-    NVFP4_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(unsigned int), s));
     if (rows == 0) return NVFP4_OK;
     const int64_t vec = dt == NVFP4_IN_FP32 ? 4 : 8;
     const int64_t total = rows * (k / vec);
     int64_t blocks = (total + 255) / 256;
     if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-    amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, rows, k, ld, dt == NVFP4_IN_FP32,
-                                                  static_cast<unsigned int*>(ws));
+    amax_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, rows, k, ld, dt == NVFP4_IN_FP32, out);
     NVFP4_CUDA_TRY(cudaGetLastError());
     return NVFP4_OK;
+}
+
+nvfp4_status launch_amax(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t k, int64_t ld, void* ws,
+                         cudaStream_t s, int sms)
+{
+    NVFP4_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(unsigned int), s));
+    return launch_amax_into(x, dt, rows, k, ld, static_cast<unsigned int*>(ws), s, sms);
 }
 
 // Multiply-shift constants for exact unsigned division by d (1 <= d < 2^31) of
@@ -883,3 +890,89 @@ nvfp4_status nvfp4_selftest_wait_timeout(long long limit_cycles, void* stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Calibrated FP8 KV cache
+// ---------------------------------------------------------------------------
+nvfp4_status nvfp4_fp8_calibrate(const void* x, nvfp4_in_dtype dt, int64_t rows, int64_t width, int64_t ld,
+                                 float* amax_inout_dev, float* scale_out_dev, void* stream)
+{
+    if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32) return fail(NVFP4_ERR_INVALID_ARG, "fp8_calibrate: bad input dtype");
+    if (rows < 0 || width <= 0 || width % 16 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "fp8_calibrate: need rows >= 0 and width a positive multiple of 16 "
+                                           "(rows=%lld width=%lld)", (long long)rows, (long long)width);
+    if (rows >= (1ll << 31) || width >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "fp8_calibrate: dimension >= 2^31");
+    if (ld < width) return fail(NVFP4_ERR_INVALID_ARG, "fp8_calibrate: ld %lld < width %lld", (long long)ld,
+                                (long long)width);
+    if (amax_inout_dev == nullptr || scale_out_dev == nullptr || (rows > 0 && x == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "fp8_calibrate: NULL pointer");
+    const int64_t esz = dt == NVFP4_IN_FP32 ? 4 : 2;
+    if (!aligned16(x) || (ld * esz) % 16 != 0 || reinterpret_cast<uintptr_t>(amax_inout_dev) % 4 ||
+        reinterpret_cast<uintptr_t>(scale_out_dev) % 4)
+        return fail(NVFP4_ERR_ALIGNMENT, "fp8_calibrate: rows must start on 16-byte boundaries");
+    DeviceState* dev = nullptr;
+    nvfp4_status st = device_state(&dev);
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = launch_amax_into(x, dt, rows, width, ld, reinterpret_cast<unsigned int*>(amax_inout_dev), s, dev->sms)) !=
+        NVFP4_OK)
+        return st;
+    fp8_scale_kernel<<<1, 32, 0, s>>>(amax_inout_dev, scale_out_dev);
+    NVFP4_CUDA_TRY(cudaGetLastError());
+    return ok();
+}
+
+nvfp4_status nvfp4_kv_cache_quantize_fp8(const void* k, const void* v, nvfp4_in_dtype dt, int64_t tokens,
+                                         int64_t width, int64_t ld_k, int64_t ld_v, const int64_t* slot_mapping,
+                                         int64_t num_slots, const float* k_scale_dev, const float* v_scale_dev,
+                                         uint8_t* k_cache, uint8_t* v_cache, int64_t cache_ld, void* stream)
+{
+    if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32)
+        return fail(NVFP4_ERR_INVALID_ARG, "kv_cache_quantize_fp8: bad input dtype");
+    if (tokens < 0 || width <= 0 || width % 16 != 0 || num_slots < 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "kv_cache_quantize_fp8: need tokens >= 0, width a positive multiple of 16 "
+                                           "and num_slots >= 0 (tokens=%lld width=%lld num_slots=%lld)",
+                    (long long)tokens, (long long)width, (long long)num_slots);
+    if (tokens * (width / 16) >= (1ll << 31))
+        return fail(NVFP4_ERR_UNSUPPORTED, "kv_cache_quantize_fp8: tokens x width / 16 >= 2^31");
+    if (ld_k < width || ld_v < width || cache_ld < width)
+        return fail(NVFP4_ERR_INVALID_ARG, "kv_cache_quantize_fp8: ld_k, ld_v and cache_ld must be >= width");
+    if (slot_mapping == nullptr && tokens > num_slots)
+        return fail(NVFP4_ERR_INVALID_ARG, "kv_cache_quantize_fp8: without a slot table token t goes to slot t, so "
+                                           "tokens (%lld) must not exceed num_slots (%lld)",
+                    (long long)tokens, (long long)num_slots);
+    if (tokens == 0) return ok();
+    if (k == nullptr || v == nullptr || k_scale_dev == nullptr || v_scale_dev == nullptr || k_cache == nullptr ||
+        v_cache == nullptr)
+        return fail(NVFP4_ERR_INVALID_ARG, "kv_cache_quantize_fp8: NULL pointer");
+    const int64_t esz = dt == NVFP4_IN_FP32 ? 4 : 2;
+    if (!aligned16(k) || !aligned16(v) || (ld_k * esz) % 16 != 0 || (ld_v * esz) % 16 != 0 || !aligned16(k_cache) ||
+        !aligned16(v_cache) || cache_ld % 16 != 0 || reinterpret_cast<uintptr_t>(slot_mapping) % 8 ||
+        reinterpret_cast<uintptr_t>(k_scale_dev) % 4 || reinterpret_cast<uintptr_t>(v_scale_dev) % 4)
+        return fail(NVFP4_ERR_ALIGNMENT, "kv_cache_quantize_fp8: rows must start on 16-byte boundaries");
+    DeviceState* dev = nullptr;
+    nvfp4_status st = device_state(&dev);
+    if (st != NVFP4_OK) return st;
+    KvParams p = {};
+    p.x[0] = k;
+    p.x[1] = v;
+    p.ld[0] = ld_k;
+    p.ld[1] = ld_v;
+    p.in_fp32 = dt == NVFP4_IN_FP32;
+    p.tokens = (uint32_t)tokens;
+    p.chunks = (uint32_t)(width / 16);
+    p.units = (uint32_t)(tokens * (width / 16));
+    p.slots = slot_mapping;
+    p.num_slots = num_slots;
+    p.scale[0] = k_scale_dev;
+    p.scale[1] = v_scale_dev;
+    p.cache[0] = k_cache;
+    p.cache[1] = v_cache;
+    p.cache_ld = cache_ld;
+    const int64_t total = 2 * (int64_t)p.units;
+    int64_t blocks = (total + kKvThreads - 1) / kKvThreads;
+    if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
+    kv_fp8_quantize_kernel<<<(unsigned)blocks, kKvThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    NVFP4_CUDA_TRY(cudaGetLastError());
+    return ok();
+}

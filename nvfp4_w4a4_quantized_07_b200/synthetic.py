@@ -134,6 +134,24 @@ def gdn_gate_params(heads: int = 48, seed: int = 9):
     return A_log.float(), dt_bias.float()
 
 
+KV_HEADS, HEAD_DIM = 4, 256   # one attention layer's K/V row: 4 KV heads x 256
+
+
+def kv_rows(tokens: int, width: int = KV_HEADS * HEAD_DIM, seed: int = 11, outlier_frac: float = 0.02,
+            outlier_gain: float = 8.0):
+    """New tokens' K and V rows (BF16, tokens x width): V ~ N(0, 1); K ~ N(0, 1)
+    with a fixed ``outlier_frac`` of its channels scaled by ``outlier_gain``
+    (keys carry a few large-magnitude channels)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    k = torch.randn(tokens, width, generator=g, dtype=torch.float32)
+    n_out = max(1, int(round(outlier_frac * width)))
+    cols = torch.randperm(width, generator=g)[:n_out]
+    k[:, cols] *= outlier_gain
+    v = torch.randn(tokens, width, generator=g, dtype=torch.float32)
+    return k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
 def mlp_glue_inputs(m: int, f: int, seed: int = 5, gate_std: float = 2.0) -> torch.Tensor:
     """A fused ``[gate | up]`` BF16 tensor of shape ``m x 2f`` (gate N(0, gate_std^2),
     up N(0, 1)), the shape of a fused gate/up GEMM output."""

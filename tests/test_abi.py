@@ -242,3 +242,30 @@ def test_gemm_gdn_argument_errors(lib):
     assert call(ptrs=(FAKE, FAKE, FAKE, ctypes.c_void_p(0x10002))) == 3
     assert call(a_col=100) == 1 and b"gemm_gdn" in lib.nvfp4_get_last_error_string()
     assert call(m=0) == 0                                # empty
+
+
+def test_fp8_kv_argument_errors(lib):
+    cal = lib.nvfp4_fp8_calibrate
+    assert cal(FAKE, 0, 8, 24, 24, FAKE, FAKE, None) == 1          # width % 16
+    assert cal(FAKE, 0, 8, 32, 16, FAKE, FAKE, None) == 1          # ld < width
+    assert cal(FAKE, 0, 8, 32, 32, None, FAKE, None) == 1          # no amax
+    assert cal(FAKE, 5, 8, 32, 32, FAKE, FAKE, None) == 1          # dtype
+    assert cal(MISALIGNED, 0, 8, 32, 32, FAKE, FAKE, None) == 3
+    kv = lib.nvfp4_kv_cache_quantize_fp8
+
+    def call(tokens=8, width=64, ld=64, slots=FAKE, num_slots=16, cache_ld=64, k=FAKE, ks=FAKE, kc=FAKE, dt=0):
+        return kv(k, FAKE, dt, tokens, width, ld, ld, slots, num_slots, ks, FAKE, kc, FAKE, cache_ld, None)
+
+    assert call(width=40) == 1                                     # width % 16
+    assert call(ld=32) == 1                                        # ld < width
+    assert call(cache_ld=48) == 1                                  # cache row shorter than width
+    assert call(num_slots=-1) == 1
+    assert call(slots=None, tokens=20) == 1                        # identity mapping past the cache
+    assert call(ks=None) == 1                                      # no scale
+    assert call(dt=3) == 1
+    assert call(k=MISALIGNED) == 3
+    assert call(cache_ld=72) == 3                                  # cache rows not 16-byte aligned
+    assert call(slots=ctypes.c_void_p(0x10004)) == 3              # slot table not 8-byte aligned
+    assert call(tokens=1 << 28, width=256) == 2                    # too many units
+    assert call(tokens=0) == 0 and call(tokens=0, k=None) == 0     # empty
+    assert call(width=40) == 1 and b"kv_cache_quantize_fp8" in lib.nvfp4_get_last_error_string()
