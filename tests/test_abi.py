@@ -269,3 +269,18 @@ def test_fp8_kv_argument_errors(lib):
     assert call(tokens=1 << 28, width=256) == 2                    # too many units
     assert call(tokens=0) == 0 and call(tokens=0, k=None) == 0     # empty
     assert call(width=40) == 1 and b"kv_cache_quantize_fp8" in lib.nvfp4_get_last_error_string()
+
+
+def test_new_bindings_refuse_host_tensors(lib):
+    """The gate and KV-cache calls run on the GPU only: host tensors are
+    rejected before any work (no CPU fallback)."""
+    import torch
+    x = torch.zeros(4, 32, dtype=torch.bfloat16)
+    one = torch.ones(1, dtype=torch.float32)
+    cache = torch.zeros(8, 32, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.fp8_calibrate(x, torch.zeros(1), one)
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.kv_cache_quantize_fp8(x, x, one, one, cache, cache.clone())
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.gemm_gdn(None, None, 0, 48, torch.zeros(48), torch.zeros(48))
