@@ -27,6 +27,11 @@
  *     with the sign bit copied from x.
  *   - two codes per byte, the even element in the low nibble.
  * Dequantisation and the GEMM are FP64 and exact up to FP64 summation.
+ *
+ * Further sections, each with its own readings: the MLP glue between the two
+ * W4A4 layers of a gated MLP (BF16 steps, as the kernels round), the Gated
+ * DeltaNet gates of the fused input projection (FP64), and the calibrated
+ * FP8 (E4M3) KV cache (FP32 product, then the E4M3 argmin).
  */
 #include <float.h>
 #include <math.h>
