@@ -10,10 +10,10 @@
 // kv_fp8_quantize_kernel quantises the new tokens' K and V rows and scatters
 // them into the cache slots a slot table names, in one launch.  It moves 2 (or
 // 4) bytes in and 1 byte out per element and does a handful of instructions
-// per element, so it is bound by HBM: one thread handles 16 consecutive
-// elements of a row (one or two 16-byte loads in flight per 16-byte store),
-// consecutive threads take consecutive pieces of a row, and the grid is a few
-// waves of resident blocks striding over the K units and then the V units.
+// per element, so it is bound by HBM: a piece is 16 consecutive elements of a
+// row (two or four 16-byte loads, one 16-byte store), consecutive threads take
+// consecutive pieces of a row, and a grid of resident blocks strides over the
+// K pieces and then the V pieces, two pieces per thread at a time.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -69,47 +69,77 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4 v, float (&f)[8])
     }
 }
 
+// Piece u (K pieces first, then V): its raw 16-byte words as loaded (two for
+// BF16, four for FP32) and where it goes.
+template <bool FP32>
+struct KvPiece {
+    uint4 raw[FP32 ? 4 : 2];
+    int tensor;
+    uint32_t t, c;
+};
+
+template <bool FP32>
+__device__ __forceinline__ void kv_load(const KvParams& p, uint32_t u, KvPiece<FP32>& x)
+{
+    x.tensor = u >= p.units;
+    const uint32_t w = u - (x.tensor ? p.units : 0);
+    x.t = w / p.chunks;
+    x.c = w - x.t * p.chunks;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x[x.tensor]) +
+                                                      ((int64_t)x.t * p.ld[x.tensor] + 16 * (int64_t)x.c) *
+                                                          (FP32 ? 4 : 2));
+#pragma unroll
+    for (int i = 0; i < (FP32 ? 4 : 2); ++i) x.raw[i] = __ldg(src + i);
+}
+
+template <bool FP32>
+__device__ __forceinline__ void kv_store(const KvParams& p, const KvPiece<FP32>& x, int64_t slot, float inv)
+{
+    if (slot < 0 || slot >= p.num_slots) return;  // padding token (or a slot past the cache)
+    float y[16];
+    if (FP32) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            y[4 * i] = __uint_as_float(x.raw[i].x);
+            y[4 * i + 1] = __uint_as_float(x.raw[i].y);
+            y[4 * i + 2] = __uint_as_float(x.raw[i].z);
+            y[4 * i + 3] = __uint_as_float(x.raw[i].w);
+        }
+    } else {
+        float lo[8], hi[8];
+        bf16x8_to_float(x.raw[0], lo);
+        bf16x8_to_float(x.raw[FP32 ? 0 : 1], hi);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            y[i] = lo[i];
+            y[8 + i] = hi[i];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(y[i], inv);
+    const uint4 out = make_uint4(fp8x4(y[0], y[1], y[2], y[3]), fp8x4(y[4], y[5], y[6], y[7]),
+                                 fp8x4(y[8], y[9], y[10], y[11]), fp8x4(y[12], y[13], y[14], y[15]));
+    *reinterpret_cast<uint4*>(p.cache[x.tensor] + slot * p.cache_ld + 16 * (int64_t)x.c) = out;
+}
+
+// Two pieces per iteration, their loads (and slot-table reads) issued before
+// either is converted, so each thread keeps 64 (BF16) or 128 (FP32) bytes in
+// flight; the scales are read once.
+template <bool FP32>
 __global__ void __launch_bounds__(kKvThreads) kv_fp8_quantize_kernel(const __grid_constant__ KvParams p)
 {
-    const uint32_t total = 2 * p.units;
-    const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += stride) {
-        const int tensor = u >= p.units;              // 0: K, 1: V
-        const uint32_t w = u - (tensor ? p.units : 0);
-        const uint32_t t = w / p.chunks, c = w - t * p.chunks;
-        const int64_t slot = p.slots != nullptr ? p.slots[t] : (int64_t)t;
-        if (slot < 0 || slot >= p.num_slots) continue;  // padding token (or a slot past the cache)
-        const float inv = fp8_inverse_scale(*p.scale[tensor]);
-        float f[16];
-        if (p.in_fp32) {
-            const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x[tensor]) +
-                                                                (int64_t)t * p.ld[tensor] + 16 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 v = __ldg(src + i);
-                f[4 * i] = v.x;
-                f[4 * i + 1] = v.y;
-                f[4 * i + 2] = v.z;
-                f[4 * i + 3] = v.w;
-            }
-        } else {
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x[tensor]) +
-                                                              (int64_t)t * p.ld[tensor] + 16 * c);
-            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-            float lo[8], hi[8];
-            bf16x8_to_float(v0, lo);
-            bf16x8_to_float(v1, hi);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                f[i] = lo[i];
-                f[8 + i] = hi[i];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(f[i], inv);
-        const uint4 out = make_uint4(fp8x4(f[0], f[1], f[2], f[3]), fp8x4(f[4], f[5], f[6], f[7]),
-                                     fp8x4(f[8], f[9], f[10], f[11]), fp8x4(f[12], f[13], f[14], f[15]));
-        *reinterpret_cast<uint4*>(p.cache[tensor] + slot * p.cache_ld + 16 * (int64_t)c) = out;
+    const uint64_t total = 2ull * p.units;  // < 2^32
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    const float inv_k = fp8_inverse_scale(*p.scale[0]), inv_v = fp8_inverse_scale(*p.scale[1]);
+    for (uint64_t u = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += 2 * stride) {
+        const bool two = u + stride < total;
+        KvPiece<FP32> a, b;
+        kv_load(p, (uint32_t)u, a);
+        if (two) kv_load(p, (uint32_t)(u + stride), b);
+        const int64_t sa = p.slots != nullptr ? p.slots[a.t] : (int64_t)a.t;
+        const int64_t sb = two ? (p.slots != nullptr ? p.slots[b.t] : (int64_t)b.t) : -1;
+        kv_store(p, a, sa, a.tensor ? inv_v : inv_k);
+        if (two) kv_store(p, b, sb, b.tensor ? inv_v : inv_k);
     }
 }
 

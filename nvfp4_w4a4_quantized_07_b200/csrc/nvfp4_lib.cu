@@ -972,7 +972,10 @@ nvfp4_status nvfp4_kv_cache_quantize_fp8(const void* k, const void* v, nvfp4_in_
     const int64_t total = 2 * (int64_t)p.units;
     int64_t blocks = (total + kKvThreads - 1) / kKvThreads;
     if (blocks > (int64_t)dev->sms * 16) blocks = (int64_t)dev->sms * 16;
-    kv_fp8_quantize_kernel<<<(unsigned)blocks, kKvThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    if (p.in_fp32)
+        kv_fp8_quantize_kernel<true><<<(unsigned)blocks, kKvThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    else
+        kv_fp8_quantize_kernel<false><<<(unsigned)blocks, kKvThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
     NVFP4_CUDA_TRY(cudaGetLastError());
     return ok();
 }
