@@ -56,6 +56,9 @@ def parse():
                     help="with --decode-case: time nvfp4_linear_decode (quantisation fused in)")
     ap.add_argument("--decode-case", default=None,
                     help="time one decode GEMM only, e.g. m16_5120x5120 (for ncu captures)")
+    ap.add_argument("--short-kernels", action="store_true",
+                    help="per-launch times of the short kernels (decode GEMMs at m=16, the FP8 KV cache at 8192 "
+                         "tokens) from back-to-back launches over rotating inputs larger than L2")
     return ap.parse_args()
 
 
@@ -759,12 +762,96 @@ def run_decode_case(args):
     return 0
 
 
+def _back_to_back_us(launches, stream, device, reps=3):
+    """Per-launch device time (us) of ``launches`` run back to back: a GPU sleep
+    of ~10 ms (longer than the host needs to enqueue them) precedes the first,
+    so the events see only the kernels and the gaps between them.  Median of
+    ``reps``."""
+    import torch
+    for f in launches[:4]:
+        f()
+    torch.cuda.synchronize(device)
+    res = []
+    for _ in range(reps):
+        torch.cuda._sleep(20_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for f in launches:
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        res.append(e0.elapsed_time(e1) * 1e3 / len(launches))
+    return statistics.median(res)
+
+
+def run_short_kernels(args):
+    """Decode GEMMs (m = 16) and the FP8 KV-cache kernel timed as 60 launches
+    back to back, each on one of several input copies that together exceed
+    twice the L2, so every launch streams its operands from HBM."""
+    import dataclasses
+
+    import torch
+
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+
+    nvbuild.build()
+    nv.load()
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(device)
+    peaks, _ = measured_peaks()
+    l2_twice = 2 * 126 * 1024 * 1024
+    out = {"method": "60 launches back to back behind a GPU sleep, inputs rotated over copies > 2x L2; "
+                     "median of 3 runs", "decode_m16": {}, "kv_cache_fp8": {}}
+    for shape, (widths, k, stds) in synthetic.DECODE_SHAPES.items():
+        mods = [synthetic.weights(n_i, k, s_i, seed=1 + i).to(device) for i, (n_i, s_i) in
+                enumerate(zip(widths, stds))]
+        fw = nv.quantize_weight(mods)
+        del mods
+        wbytes = fw.q.numel() + fw.sf.numel()
+        copies = [fw] + [dataclasses.replace(fw, q=fw.q.clone(), sf=fw.sf.clone())
+                         for _ in range(max(1, -(-l2_twice // wbytes)) - 1)]
+        a, _ = synthetic.activations(16, k, seed=0, n_outliers=0)
+        aq = nv.quantize_act(a.to(device))
+        c = torch.empty((16, fw.n), dtype=torch.bfloat16, device=device)
+        launches = [(lambda w=copies[i % len(copies)]: nv.gemm(aq, w, out=c)) for i in range(60)]
+        us = _back_to_back_us(launches, stream, device)
+        nbytes = wbytes + aq.q.numel() + aq.sf.numel() + c.numel() * 2
+        out["decode_m16"][shape] = {"us": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
+                                    "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                                    "weight_copies": len(copies)}
+        del copies, fw
+    tokens = 8192
+    sets = []
+    for r in range(6):
+        k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens, seed=11 + r))
+        ks = torch.empty(1, dtype=torch.float32, device=device)
+        vs = torch.empty(1, dtype=torch.float32, device=device)
+        nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
+        nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
+        slots = torch.randperm(2 * tokens, generator=torch.Generator().manual_seed(r))[:tokens].to(device)
+        kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
+        sets.append((k_rows, v_rows, ks, vs, kc, torch.empty_like(kc), slots))
+    launches = [(lambda s_=sets[i % len(sets)]: nv.kv_cache_quantize_fp8(*s_)) for i in range(60)]
+    us = _back_to_back_us(launches, stream, device)
+    k0 = sets[0][0]
+    nbytes = 2 * k0.numel() * (k0.element_size() + 1) + tokens * 8
+    out["kv_cache_fp8"][f"tokens{tokens}_width{k0.shape[1]}"] = {
+        "us": us, "GB/s": nbytes / (us * 1e-6) / 1e9, "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+        "input_copies": len(sets)}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.decode_case:
         return run_decode_case(args)
+    if args.short_kernels:
+        return run_short_kernels(args)
     if args.probe_peaks:
         return run_probe_peaks(args)
     if args.glue_case:
