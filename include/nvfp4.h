@@ -103,10 +103,12 @@ NVFP4_API int64_t nvfp4_sf_offset(int64_t row, int64_t kblock, int64_t k);
 NVFP4_API size_t nvfp4_quant_workspace_size(void);
 
 /* Workspace bytes nvfp4_gemm needs for this shape and kernel choice: 0 for
- * the large-M kernels; for the decode kernel (m <= 64) 2 KiB of per-CTA flags
- * plus one 256-column FP32 partial tile of 16, 32 or 64 rows per CTA slot
- * (256 slots): 4, 8 or 16 MiB.  The workspace needs no
- * initialisation, but two calls that may run concurrently must not share one. */
+ * the large-M kernels; for the decode kernel (m <= 64) one partial tile of
+ * 16, 32 or 64 rows x 128 columns per CTA slot (160 slots), each value an
+ * 8-byte word (FP32 and a 32-bit tag): 2.5, 5 or 10 MiB.  The workspace needs no
+ * initialisation, but two calls that may run concurrently must not share one
+ * (consecutive calls on one stream may share it: a decode kernel touches the
+ * workspace only after the previous kernel in the stream has completed). */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags);
 
 /* ------------------------------------------------------------------------
@@ -177,8 +179,13 @@ NVFP4_API nvfp4_status nvfp4_quantize_act(const void* a, nvfp4_in_dtype dt, int6
  *   workspace         device, >= nvfp4_gemm_workspace_size(m, n, k, flags)
  *                     bytes, 16-byte aligned (may be NULL when that is 0).
  *                     The decode kernel passes partial tiles between its CTAs
- *                     through it; it is launched cooperatively (all CTAs
- *                     resident), one CTA per SM.
+ *                     through it (one CTA per SM).  It is launched with
+ *                     programmatic dependent launch: its CTAs may start, and
+ *                     load weights, while the previous kernel in the stream
+ *                     is still running, and touch activations, scales,
+ *                     workspace and output only after that kernel has
+ *                     completed.  Back-to-back decode GEMMs thus overlap the
+ *                     next weight stream with the previous GEMM's tail.
  *   flags             NVFP4_GEMM_* kernel choice.
  * Shapes: m >= 1, n a multiple of 16, k a multiple of 32, all < 2^31.
  * The BF16 output is the round-to-nearest-even BF16 of the FP32 output of the
@@ -323,8 +330,8 @@ NVFP4_API nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int
  * plain C host with no device allocator; and for callers that must not
  * allocate in the middle of a step, because a device allocation can block
  * until the device is idle or fail when memory is tight.  The call allocates
- * nothing.  The kernel's scratch (one flag per CTA slot and one FP32 partial
- * tile per CTA slot) lives in a fixed array of NVFP4_NOALLOC_SCRATCH_BYTES
+ * nothing.  The kernel's scratch (one tagged FP32 partial tile per CTA
+ * slot) lives in a fixed array of NVFP4_NOALLOC_SCRATCH_BYTES
  * bytes of device memory that the library reserves on each device it is
  * loaded on.
  *
@@ -337,14 +344,13 @@ NVFP4_API nvfp4_status nvfp4_silu_mul_quantize(const void* g, const void* u, int
  *   the array's device address and sets the kernels' attributes.  Make that
  *   first call before any stream capture begins.
  * Sharing: every call on a device uses the same array.  Nothing in it has to
- *   be zero when a call starts: a CTA's flag is compared with a value fresh to
- *   each call, and every partial tile is written before it is read in the
- *   same call.  Two calls that overlap in time on one device (different
+ *   be zero when a call starts: every partial word carries a tag fresh to each
+ *   call, and a reader waits for words with its own call's tag.  Two calls that overlap in time on one device (different
  *   streams, or threads without ordering) race on the array and give wrong
  *   results; order them (one stream, or events).
  * ---------------------------------------------------------------------- */
 #define NVFP4_NOALLOC_MAX_M 16
-#define NVFP4_NOALLOC_SCRATCH_BYTES (2048 + 256 * 16 * 256 * 4) /* 4 MiB + 2 KiB */
+#define NVFP4_NOALLOC_SCRATCH_BYTES (160 * 16 * 128 * 8) /* 2.5 MiB */
 NVFP4_API nvfp4_status nvfp4_gemm_decode_noalloc(const uint8_t* a_q, const uint8_t* a_sf, const float* act_scale_dev,
                                        const uint8_t* w_q, const uint8_t* w_sf, int64_t m, int64_t n, int64_t k,
                                        const nvfp4_segment* segs, int nsegs, void* c, nvfp4_out_dtype odt,

@@ -21,8 +21,8 @@
 //  * gemm_decode.cuh: gemm_decode_kernel, small M (<= 64 tokens), bound by
 //    streaming the weight.  Stream-K: the (256-column tile, 256-deep k-tile)
 //    units are split evenly over one CTA per SM; a tile whose k-range spans
-//    several CTAs is finished by the CTA holding its first k-tile, which adds
-//    the others' FP32 partials in CTA order, so the result is deterministic.
+//    several CTAs is reduced by all of them, each summing a column slice of
+//    the FP32 partials in CTA order, so the result is deterministic.
 #pragma once
 
 #include <cuda.h>
@@ -56,8 +56,8 @@ struct GemmParams {
     // decode kernel (stream-K): work units = w_tiles x k_tiles, split evenly
     // over `ctas` co-resident CTAs; partial tiles meet in `ws`
     int units, ctas;
-    uint8_t* ws;                // [256] uint64 flags, then [256][BT][256] FP32 partial tiles
-    unsigned long long epoch;   // this call's flag value
+    uint8_t* ws;                // [MAX_CTAS][2][BT][256] tagged partial-tile words
+    unsigned long long epoch;   // this call's value; its low 32 bits tag the partial words
     // decode kernel with the activation quantisation fused in: the raw
     // activations (act_scale == nullptr: dynamic scale amax/2688, computed by
     // every CTA; CTA 0 writes it to act_scale_out when that is given)

@@ -8,61 +8,88 @@
 namespace nvfp4 {
 
 // ===========================================================================
-// Decode kernel (M <= 64): stream-K over 256-column output tiles.
+// Decode kernel (M <= 64): stream-K over 128-column output tiles.
 //
-// Small M is pure weight streaming, and on this hardware every TMA / bulk
-// copy instruction and every block-scaled MMA has a fixed issue cost (~150
-// cycles) whatever its size.  So the kernel keeps both large: the tokens are
-// the MMA's M side (a 128-row operand of which only the first M rows are
-// loaded and stored -- the rest is never read back), 256 weight rows its N
-// side, 32 KB weight tiles per stage.  The (256-column tile, 256-deep k-tile)
-// work units are split evenly over exactly one CTA per SM (a cooperative
-// launch keeps them all resident).  A tile whose k-tiles span several CTAs is
-// finished by the CTA holding its first k-tile: the others reach their part of
-// it first, leave FP32 partials in the workspace and publish them with this
-// call's epoch value; the owner adds them in CTA order, so the result does not
-// depend on timing.
+// Small M is pure weight streaming.  What a launch costs beyond the weight
+// bytes is fixed: getting the CTAs onto the SMs, the first HBM round trip, and
+// the hand-off of tiles whose K range is split between CTAs.  The kernel hides
+// the first two under the previous kernel in the stream and keeps the third
+// short:
 //
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocation, 4..7
-// epilogue (TMEM quadrants 0-3 = token rows 0..127), 8..11 scale staging.
-// TMEM: accumulator [0, 256), four 48-column scale slots [256, 448).
+//  * Programmatic dependent launch.  Every CTA lets the next kernel launch as
+//    soon as its barriers exist.  Before it waits for the previous kernel to
+//    complete it only touches weights (which no earlier kernel writes): it
+//    fills its shared-memory ring with weight tiles.  Activations, the
+//    activation scale, TMEM and every global write come after that wait.
+//  * Few, large copies: a stage is two 256-deep k-tiles of one tile (32 KB of
+//    weights), brought in by four copy instructions (weights, their scale
+//    atoms, token rows, token scales; the two k-tiles of a 128-byte-wide
+//    operand come as one 3-D box when K is a multiple of 256) -- the copy
+//    engine's issue rate, not HBM, limits rings of many small copies.
+//  * Stream-K: the (tile, k-tile) units are split evenly over one CTA per SM.
+//    A tile whose k-tiles span several CTAs is finished by the CTA holding its
+//    first k-tile (the "owner"), which reaches its part last (it ends its
+//    range); the others reach their part first (it starts their range),
+//    leave the FP32 partial in the workspace -- every value paired with a
+//    32-bit tag fresh to this call in one 8-byte word, so no flag or fence is
+//    needed -- and exit.  The owner loads the partials (waiting for their
+//    tags) and adds them in CTA order, so the result does not depend on
+//    timing.  Contributors leave early, which frees their SMs for the next
+//    kernel's CTAs.
+//
+// The tokens are the MMA's M side: a 128-row operand of which only the first
+// BT rows are loaded (the rest reads whatever follows in shared memory; those
+// accumulator rows are never read back).  128 weight rows are its N side, so a
+// split tile's partial is m x 128 and an owner adds few of them.  Two TMEM
+// accumulators let the MMAs of the next segment run while the epilogue drains
+// the last one.
+//
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocation (and, with the
+// activation quantisation fused in, 2..3 quantise), 4..7 epilogue (TMEM lane
+// quadrants 0..3 = token rows 0..127), 8..11 scale staging; an owner's twelve
+// warps all take part in its finish.
+// TMEM: accumulators [0, 128) and [128, 256), four 64-column scale slots
+// [256, 512); allocated after the dependency wait.
 // ===========================================================================
 namespace decode {
-constexpr int BN = 256;                      // output columns (weight rows) per tile = the MMA's N
-constexpr int BK_BYTES = 128;
-constexpr int KSTEPS = 4;
+constexpr int BN = 128;                      // output columns (weight rows) per tile = the MMA's N
+constexpr int KT_BYTES = 128;                // one k-tile: 256 FP4 values = 128 bytes of a row
+constexpr int KT_PER_STAGE = 2;
+constexpr int KSTEPS = 4;                    // MMAs (K = 64) per k-tile
 constexpr int THREADS = 384;
-constexpr int B_STAGE = BN * BK_BYTES;       // 32 KB of weights
-constexpr int SFA_STAGE = 4 * 512;           // token scale atoms (one 128-row block)
-constexpr int SFB_STAGE = 2 * 4 * 512;       // weight scale atoms (two 128-row blocks)
+constexpr int W_KT = BN * KT_BYTES;          // 16 KB of weights per k-tile
+constexpr int W_STAGE = KT_PER_STAGE * W_KT;
+constexpr int SF_KT = KSTEPS * 512;          // scale atoms of one 128-row block per k-tile
+constexpr int SF_STAGE = KT_PER_STAGE * SF_KT;
 constexpr int SF_SLOTS = 4;
+constexpr int SF_SLOT = 64;                  // per stage: A (8 k-steps x 4 columns), then B (8 x 4)
 constexpr int ACC_PITCH = BN + 4;            // floats per staged accumulator row: float4 access is conflict-free
 constexpr int TMEM_COLS = 512;
-constexpr int SF_COL = 256;
-constexpr int SF_SLOT = 48;                  // 16 (tokens: 4 k-steps x 4) + 32 (weights: 4 x 8)
-constexpr int MAX_CTAS = 256;
-constexpr int FLAGS_BYTES = MAX_CTAS * 8;
+constexpr int SF_COL = 2 * BN;
+constexpr int MAX_CTAS = 160;                // grid cap (one CTA per SM); sizes the workspace
 static_assert(SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "TMEM budget");
 
 // Shared-memory plan for BT token rows.  The A stage holds only the BT loaded
-// rows; the M = 128 MMA reads 16 KB from its start, running on into the next
-// buffers, and the accumulator rows that come from those bytes are never read.
+// rows of each k-tile; the M = 128 MMA reads 16 KB from the start of a
+// k-tile's rows, running on into the next buffers, and the accumulator rows
+// that come from those bytes are never read.
 template <int BT>
 struct Cfg {
-    static constexpr int STAGES = BT >= 64 ? 3 : (BT >= 32 ? 4 : 5);
-    static constexpr int A_STAGE = BT * BK_BYTES;
+    static constexpr int STAGES = BT >= 64 ? 3 : 4;
+    static constexpr int A_KT = BT * KT_BYTES;
+    static constexpr int A_STAGE = KT_PER_STAGE * A_KT;
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
-    static constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
-    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-    static constexpr int OFF_ACC = OFF_SFB + STAGES * SFB_STAGE;
+    static constexpr int OFF_W = OFF_A + STAGES * A_STAGE;
+    static constexpr int OFF_SFA = OFF_W + STAGES * W_STAGE;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SF_STAGE;
+    static constexpr int OFF_ACC = OFF_SFB + STAGES * SF_STAGE;
     static constexpr int OFF_BAR = OFF_ACC + BT * ACC_PITCH * 4;
-    // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full, acc_empty, drain, sga_ready
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 4;
+    // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full[2], acc_empty[2], drain, sga_ready
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 6;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, verdicts, s_ga, amax partials
     static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
-    static_assert(A_STAGE % 1024 == 0, "SW128 stages are 1 KB aligned");
-    static_assert(OFF_A + (STAGES - 1) * A_STAGE + 128 * BK_BYTES <= OFF_MISC, "MMA A reads stay in the buffer");
+    static_assert(A_KT % 1024 == 0, "SW128 operand tiles are 1 KB aligned");
+    static_assert(OFF_A + STAGES * A_STAGE - A_KT + 128 * KT_BYTES <= OFF_MISC, "MMA A reads stay in the buffer");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -72,19 +99,27 @@ __device__ __forceinline__ int cta_of_unit(int64_t u, int units, int ctas)
 {
     return (int)(((u + 1) * ctas + units - 1) / units) - 1;
 }
+
+// The stage starting at unit u of a CTA's range [u_begin, u_end): tile nb,
+// k-tiles [kt, kt + nkt) (at most two, never crossing a tile), whether it
+// opens and whether it closes a segment (the CTA's run of units in one tile).
+struct Stage {
+    int nb, kt, nkt;
+    bool first, last;
+};
+
+__device__ __forceinline__ Stage stage_at(int64_t u, int64_t u_begin, int64_t u_end, int k_tiles)
+{
+    Stage s;
+    s.nb = (int)(u / k_tiles);
+    s.kt = (int)(u - (int64_t)s.nb * k_tiles);
+    const int64_t seg_stop = min(u_end, (int64_t)(s.nb + 1) * k_tiles);
+    s.nkt = (int)min((int64_t)KT_PER_STAGE, seg_stop - u);
+    s.first = u == u_begin || s.kt == 0;
+    s.last = u + s.nkt == seg_stop;
+    return s;
+}
 }  // namespace decode
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p)
-{
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v)
-{
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
 // Scale 4 consecutive output columns of one row by s_ga * s_gw[seg] and store
 // them (4 columns never straddle a segment: boundaries are multiples of 16).
@@ -104,21 +139,83 @@ __device__ __forceinline__ void store4_scaled(const GemmParams& p, int row, int 
     }
 }
 
+// Partial-tile words: (tag << 32) | FP32 bits, written and read as morally
+// strong 8-byte accesses, so a word is either wholly this call's or not.
+__device__ __forceinline__ void st_tagged4(unsigned long long* dst, float4 v, uint32_t tag)
+{
+    const unsigned long long t = (unsigned long long)tag << 32;
+    asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(dst), "l"(t | __float_as_uint(v.x)),
+                 "l"(t | __float_as_uint(v.y))
+                 : "memory");
+    asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(dst + 2), "l"(t | __float_as_uint(v.z)),
+                 "l"(t | __float_as_uint(v.w))
+                 : "memory");
+}
+
+// Four tagged words: load them, then (after any number of other loads are
+// in flight) check that all carry this call's tag and unpack the values.
+struct Tagged4 {
+    unsigned long long w[4];
+};
+
+__device__ __forceinline__ void ld_tagged4(const unsigned long long* src, Tagged4& t)
+{
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(t.w[0]), "=l"(t.w[1]) : "l"(src) : "memory");
+    asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];" : "=l"(t.w[2]), "=l"(t.w[3]) : "l"(src + 2) : "memory");
+}
+
+__device__ __forceinline__ bool tagged4_ok(const Tagged4& t, uint32_t tag)
+{
+    return (uint32_t)(t.w[0] >> 32) == tag && (uint32_t)(t.w[1] >> 32) == tag && (uint32_t)(t.w[2] >> 32) == tag &&
+           (uint32_t)(t.w[3] >> 32) == tag;
+}
+
+__device__ __forceinline__ float4 tagged4_value(const Tagged4& t)
+{
+    return make_float4(__uint_as_float((uint32_t)t.w[0]), __uint_as_float((uint32_t)t.w[1]),
+                       __uint_as_float((uint32_t)t.w[2]), __uint_as_float((uint32_t)t.w[3]));
+}
+
+// Copy k-tiles [kt, kt + nkt) of a 128-byte-wide operand (rows starting at
+// `row`): one 3-D box for two k-tiles when the 3-D map exists (K a multiple of
+// 256), else one 2-D box per k-tile.  Tiles of the stage sit `tile_bytes` apart.
+__device__ __forceinline__ void load_ktiles(uint8_t* dst, const CUtensorMap* map2, const CUtensorMap* map3, bool use3,
+                                            uint64_t* bar, int kt, int nkt, int row, int tile_bytes)
+{
+    if (use3 && nkt == 2) {
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+            "l"(map3), "r"(0), "r"(row), "r"(kt), "r"(smem_u32(bar))
+            : "memory");
+    } else {
+        for (int j = 0; j < nkt; ++j)
+            tma_load_2d(dst + j * tile_bytes, map2, bar, (kt + j) * decode::KT_BYTES, row);
+    }
+}
+
+// The decode kernel's tensor maps: 2-D maps of the token rows (box 128 bytes x
+// BT rows) and of the weight (128 bytes x 128 rows), and 3-D views
+// {128 bytes, rows, K / 256} of the same buffers (boxes two k-tiles deep),
+// used when K is a multiple of 256.
+struct DecodeMaps {
+    CUtensorMap a, w, a3, w3;
+};
+
 // FQ: the activation quantisation is fused in.  Warps 2 and 3 then quantise
-// the stage's BT x 256 slice of the raw activations straight into the A stage
-// (the 128-byte-swizzled layout the TMA would have written) and the scale
-// atoms into the scale stage, with the same block arithmetic as
+// each stage's BT x 256 slices of the raw activations straight into the A
+// stage (the 128-byte-swizzled layout the TMA would have written) and the
+// scale atoms into the scale stage, with the same block arithmetic as
 // quantize_kernel, so the result is bit-identical to quantising first.
 template <int BT, bool FQ>
 __global__ void __launch_bounds__(decode::THREADS, 1)
-    gemm_decode_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-                       const __grid_constant__ GemmParams p)
+    gemm_decode_kernel(const __grid_constant__ DecodeMaps maps, const __grid_constant__ GemmParams p)
 {
     using namespace decode;
     using C = Cfg<BT>;
     constexpr int STAGES = C::STAGES;
-    constexpr int A_STAGE = C::A_STAGE;
-    constexpr int OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_SFA = C::OFF_SFA, OFF_SFB = C::OFF_SFB;
+    constexpr int A_KT = C::A_KT, A_STAGE = C::A_STAGE;
+    constexpr int OFF_A = C::OFF_A, OFF_W = C::OFF_W, OFF_SFA = C::OFF_SFA, OFF_SFB = C::OFF_SFB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -126,15 +223,14 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
     uint64_t* sf_ready = empty + STAGES;
     uint64_t* sf_free = sf_ready + SF_SLOTS;
     uint64_t* acc_full = sf_free + SF_SLOTS;
-    uint64_t* acc_empty = acc_full + 1;
-    uint64_t* drain = acc_empty + 1;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
     uint64_t* sga_ready = drain + 1;   // FQ: the activation scale is in s_ga_smem
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-    volatile int* acc_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);    // acc_full verdict
-    volatile int* peers_bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8); // a peer wait ran out
+    volatile int* bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);        // a wait ran out
+    volatile int* verdict = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);    // epilogue barrier verdict
     volatile float* s_ga_smem = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 12); // FQ: the scale used
     volatile float* amax_part = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 16); // FQ: [2]
-    volatile int* sga_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 24);         // FQ: sga_ready verdict
     float* acc_stage = reinterpret_cast<float*>(smem + C::OFF_ACC);
 
     const int warp = threadIdx.x >> 5;
@@ -143,10 +239,16 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
     const int64_t u_begin = (int64_t)cta * p.units / p.ctas;
     const int64_t u_end = (int64_t)(cta + 1) * p.units / p.ctas;
     const int k_tiles = p.k_tiles;
+    const bool use3 = p.k % 256 == 0;
+    // contributor c's partial tile: BT x BN tagged words at parts + c BT BN
+    unsigned long long* parts = reinterpret_cast<unsigned long long*>(p.ws);
+    const uint32_t tag = (uint32_t)p.epoch;
 
     if (warp == 0 && lane == 0) {
-        prefetch_tensor_map(&tmap_a);
-        prefetch_tensor_map(&tmap_w);
+        prefetch_tensor_map(&maps.a);
+        prefetch_tensor_map(&maps.w);
+        prefetch_tensor_map(&maps.a3);
+        prefetch_tensor_map(&maps.w3);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], FQ ? 3 : 1);    // FQ: the producer and the two quantiser warps
             mbar_init(&empty[s], 1);
@@ -155,63 +257,106 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
             mbar_init(&sf_ready[i], 4);
             mbar_init(&sf_free[i], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
         mbar_init(drain, 1);
         mbar_init(sga_ready, 1);
-        *peers_bad = 0;
-        *acc_ok = 0;
+        *bad = 0;
         fence_mbarrier_init();
     }
-    if (warp == 2) {
-        tmem_alloc(tmem_ptr, TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_ptr;
+    // The next kernel in the stream may launch now; it waits for this one
+    // before it reads or writes anything this one may write.
+    if (threadIdx.x == 0) launch_dependents();
+
+    uint32_t tmem_base = 0;
+    if (warp != 0) {
+        // Everything but the producer waits for the previous kernel here; then
+        // TMEM, which that kernel may have held on this SM, is free.
+        dependency_wait();
+        if (warp == 2) {
+            tmem_alloc(tmem_ptr, TMEM_COLS);
+            tmem_relinquish();
+        }
+        if (warp != 3) {
+            tc_fence_before();
+            asm volatile("bar.sync 4, 320;" ::: "memory");   // warps 1, 2, 4..11
+            tc_fence_after();
+            tmem_base = *tmem_ptr;
+        }
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
             bool ok = true;
-            int nb = (int)(u_begin / k_tiles), kt = (int)(u_begin - (int64_t)nb * k_tiles);
-            for (int64_t u = u_begin; u < u_end; ++u) {
+            // Pass 1 (before the dependency wait): the weights and weight scales
+            // of the first ring pass.  Without FQ each of these stages arrives
+            // later, with its activation copies.
+            int64_t u = u_begin;
+            int pre = 0;
+            for (; u < u_end && pre < STAGES; ++pre) {
+                const Stage st = stage_at(u, u_begin, u_end, k_tiles);
+                const int nsf = min(KSTEPS * st.nkt, p.katoms - st.kt * KSTEPS);
+                const uint32_t wbytes = (uint32_t)(st.nkt * W_KT + nsf * 512);
+                if (FQ)
+                    mbar_arrive_expect_tx(&full[pre], wbytes);
+                else
+                    mbar_expect_tx(&full[pre], wbytes);
+                load_ktiles(smem + OFF_W + pre * W_STAGE, &maps.w, &maps.w3, use3, &full[pre], st.kt, st.nkt,
+                            st.nb * BN, W_KT);
+                bulk_load(smem + OFF_SFB + pre * SF_STAGE, p.w_sf + ((int64_t)st.nb * p.katoms + st.kt * KSTEPS) * 512,
+                          (uint32_t)nsf * 512u, &full[pre]);
+                u += st.nkt;
+            }
+            dependency_wait();
+            if (!FQ) {
+                // Pass 2: the activation side of those stages.
+                int64_t v = u_begin;
+                for (int s = 0; s < pre; ++s) {
+                    const Stage st = stage_at(v, u_begin, u_end, k_tiles);
+                    const int nsf = min(KSTEPS * st.nkt, p.katoms - st.kt * KSTEPS);
+                    mbar_arrive_expect_tx(&full[s], (uint32_t)(st.nkt * A_KT + nsf * 512));
+                    load_ktiles(smem + OFF_A + s * A_STAGE, &maps.a, &maps.a3, use3, &full[s], st.kt, st.nkt, 0, A_KT);
+                    bulk_load(smem + OFF_SFA + s * SF_STAGE, p.a_sf + (int64_t)st.kt * KSTEPS * 512,
+                              (uint32_t)nsf * 512u, &full[s]);
+                    v += st.nkt;
+                }
+            }
+            // Steady state: whole stages as the ring frees them.
+            int stage = 0;
+            uint32_t phase = 1;
+            while (u < u_end) {
+                const Stage st = stage_at(u, u_begin, u_end, k_tiles);
                 if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
                     ok = false;
                     break;
                 }
-                const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
-                const uint32_t sf_bytes = (uint32_t)nks * 512u;
-                const bool rb1 = 2 * nb + 1 < p.w_rowblocks;
-                if (FQ) {
-                    mbar_arrive_expect_tx(&full[stage], B_STAGE + sf_bytes * (rb1 ? 2u : 1u));
-                } else {
-                    mbar_arrive_expect_tx(&full[stage], BT * BK_BYTES + B_STAGE + sf_bytes * (rb1 ? 3u : 2u));
-                    tma_load_2d(smem + OFF_A + stage * A_STAGE, &tmap_a, &full[stage], kt * BK_BYTES, 0);
-                    bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_sf + (int64_t)kt * KSTEPS * 512, sf_bytes,
-                              &full[stage]);
+                const int nsf = min(KSTEPS * st.nkt, p.katoms - st.kt * KSTEPS);
+                const uint32_t bytes =
+                    (uint32_t)(st.nkt * W_KT + nsf * 512 + (FQ ? 0 : st.nkt * A_KT + nsf * 512));
+                mbar_arrive_expect_tx(&full[stage], bytes);
+                load_ktiles(smem + OFF_W + stage * W_STAGE, &maps.w, &maps.w3, use3, &full[stage], st.kt, st.nkt,
+                            st.nb * BN, W_KT);
+                bulk_load(smem + OFF_SFB + stage * SF_STAGE,
+                          p.w_sf + ((int64_t)st.nb * p.katoms + st.kt * KSTEPS) * 512, (uint32_t)nsf * 512u,
+                          &full[stage]);
+                if (!FQ) {
+                    load_ktiles(smem + OFF_A + stage * A_STAGE, &maps.a, &maps.a3, use3, &full[stage], st.kt, st.nkt, 0,
+                                A_KT);
+                    bulk_load(smem + OFF_SFA + stage * SF_STAGE, p.a_sf + (int64_t)st.kt * KSTEPS * 512,
+                              (uint32_t)nsf * 512u, &full[stage]);
                 }
-                tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmap_w, &full[stage], kt * BK_BYTES, nb * BN);
-                bulk_load(smem + OFF_SFB + stage * SFB_STAGE,
-                          p.w_sf + ((int64_t)(2 * nb) * p.katoms + kt * KSTEPS) * 512, sf_bytes, &full[stage]);
-                if (rb1)
-                    bulk_load(smem + OFF_SFB + stage * SFB_STAGE + 2048,
-                              p.w_sf + ((int64_t)(2 * nb + 1) * p.katoms + kt * KSTEPS) * 512, sf_bytes,
-                              &full[stage]);
+                u += st.nkt;
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
-                if (++kt == k_tiles) {
-                    kt = 0;
-                    ++nb;
-                }
             }
             if (!ok) {
+                *bad = 1;
                 const long long t0 = clock64();
                 while (clock64() - t0 < kWaitCycles / 64) {
                 }
@@ -222,33 +367,37 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_nvf4(128, BN);
-            int stage = 0, slot = 0;
-            uint32_t slot_phase = 0, segs = 0;
-            bool ok = true, first = true;
-            int kt = (int)(u_begin % k_tiles);
-            for (int64_t u = u_begin; u < u_end && ok; ++u) {
-                if (u == u_begin || kt == 0) {
-                    // a new segment: the accumulator has been drained
-                    if (!mbar_wait(acc_empty, (segs & 1) ^ 1, kStatusTimeoutAccum)) {
+            int stage = 0, slot = 0, seg = 0;
+            uint32_t slot_phase = 0;
+            bool ok = true;
+            for (int64_t u = u_begin; u < u_end;) {
+                const Stage st = stage_at(u, u_begin, u_end, k_tiles);
+                const int b = seg & 1;
+                if (st.first) {
+                    // a new segment: this accumulator's previous segment has been drained
+                    if (!mbar_wait(&acc_empty[b], ((seg >> 1) & 1) ^ 1, kStatusTimeoutAccum)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    first = true;
                 }
                 if (!mbar_wait(&sf_ready[slot], slot_phase, kStatusTimeoutFull)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int nks = min(KSTEPS, p.katoms - kt * KSTEPS);
+                const int nks = min(KSTEPS * st.nkt, p.katoms - st.kt * KSTEPS);
                 const uint32_t sf_col = tmem_base + SF_COL + slot * SF_SLOT;
+                const uint32_t acc = tmem_base + b * BN;
                 const uint64_t adesc = desc_kmajor_sw128(smem + OFF_A + stage * A_STAGE);
-                const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_B + stage * B_STAGE);
-                for (int ks = 0; ks < nks; ++ks)
-                    mma_nvf4(tmem_base, adesc + 2 * ks, bdesc + 2 * ks, idesc, !(first && ks == 0), sf_col + 4 * ks,
-                             sf_col + 16 + 8 * ks);
-                first = false;
+                const uint64_t bdesc = desc_kmajor_sw128(smem + OFF_W + stage * W_STAGE);
+                for (int ks = 0; ks < nks; ++ks) {
+                    // k-tile j = ks / 4 of the stage, 64 FP4 values (32 bytes, +2 in the
+                    // descriptor's 16-byte units) per k-step inside it
+                    const int j = ks >> 2, q = ks & 3;
+                    mma_nvf4(acc, adesc + (uint64_t)((j * A_KT) >> 4) + 2 * q, bdesc + (uint64_t)((j * W_KT) >> 4) + 2 * q,
+                             idesc, !(st.first && ks == 0), sf_col + 4 * ks, sf_col + 32 + 4 * ks);
+                }
                 mma_commit(&empty[stage]);
                 mma_commit(&sf_free[slot]);
                 if (++stage == STAGES) stage = 0;
@@ -256,13 +405,14 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                     slot = 0;
                     slot_phase ^= 1;
                 }
-                if (u == u_end - 1 || kt == k_tiles - 1) {
-                    mma_commit(acc_full);
-                    ++segs;
+                if (st.last) {
+                    mma_commit(&acc_full[b]);
+                    ++seg;
                 }
-                if (++kt == k_tiles) kt = 0;
+                u += st.nkt;
             }
             if (!ok) {
+                *bad = 1;
                 mma_commit(drain);
                 mbar_wait(drain, 0, kStatusTimeoutDrain, kWaitCycles / 8);
             }
@@ -297,81 +447,87 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
         }
         int stage = 0;
         uint32_t phase = 0;
-        int kt = (int)(u_begin % k_tiles);
         const int64_t esz = p.a_fp32 ? 4 : 2;
-        // Each thread owns BT / 8 chunks (row r, 32 columns) of a stage, taken two
-        // at a time: all loads of a pair are issued before any arithmetic, and
-        // the first pair's loads before the wait for the stage buffer (they do
-        // not need it), so the L2 round trip overlaps the wait.
+        // Each thread owns BT / 8 chunks (row r, 32 columns) of each k-tile of a
+        // stage, taken two at a time: all loads of a pair are issued before any
+        // arithmetic, and the first pair's loads before the wait for the stage
+        // buffer (they do not need it), so the L2 round trip overlaps the wait.
         constexpr int CPT = BT / 8;
         constexpr int CB = CPT < 2 ? CPT : 2;
-        for (int64_t u = u_begin; u < u_end; ++u) {
-            uint8_t* adst = smem + OFF_A + stage * A_STAGE;
-            uint8_t* sdst = smem + OFF_SFA + stage * SFA_STAGE;
+        for (int64_t u = u_begin; u < u_end;) {
+            const Stage st = stage_at(u, u_begin, u_end, k_tiles);
             bool waited = false, ok = true;
+            for (int h = 0; h < st.nkt && ok; ++h) {
+                const int kt = st.kt + h;
+                uint8_t* adst = smem + OFF_A + stage * A_STAGE + h * A_KT;
+                uint8_t* sdst = smem + OFF_SFA + stage * SF_STAGE + h * SF_KT;
 #pragma unroll
-            for (int b0 = 0; b0 < CPT; b0 += CB) {
-                uint4 raw[CB][8];
-                bool l0[CB], l1[CB];
+                for (int b0 = 0; b0 < CPT; b0 += CB) {
+                    uint4 raw[CB][8];
+                    bool l0[CB], l1[CB];
 #pragma unroll
-                for (int j = 0; j < CB; ++j) {
-                    const int it = qt + 64 * (b0 + j);
-                    const int r = it >> 3, c = it & 7;
-                    const int64_t k0 = (int64_t)kt * 256 + c * 32;
-                    l0[j] = r < p.m && k0 < p.k;
-                    l1[j] = r < p.m && k0 + 16 < p.k;
-                    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.a_in) +
-                                                                      ((int64_t)r * p.lda + k0) * esz);
-                    const int words = p.a_fp32 ? 8 : 4;   // 16-byte words per 32 elements
+                    for (int j = 0; j < CB; ++j) {
+                        const int it = qt + 64 * (b0 + j);
+                        const int r = it >> 3, c = it & 7;
+                        const int64_t k0 = (int64_t)kt * 256 + c * 32;
+                        l0[j] = r < p.m && k0 < p.k;
+                        l1[j] = r < p.m && k0 + 16 < p.k;
+                        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.a_in) +
+                                                                          ((int64_t)r * p.lda + k0) * esz);
+                        const int words = p.a_fp32 ? 8 : 4;   // 16-byte words per 32 elements
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) {
-                        const bool lv = (w < words / 2) ? l0[j] : l1[j];
-                        raw[j][w] = (w < words && lv) ? __ldg(src + w) : make_uint4(0, 0, 0, 0);
-                    }
-                }
-                if (!waited) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
-                        ok = false;
-                        break;
-                    }
-                    waited = true;
-                }
-#pragma unroll
-                for (int j = 0; j < CB; ++j) {
-                    const int it = qt + 64 * (b0 + j);
-                    const int r = it >> 3, c = it & 7;
-                    float v0[16], v1[16];
-                    if (p.a_fp32) {
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            v0[4 * w] = __uint_as_float(raw[j][w].x);
-                            v0[4 * w + 1] = __uint_as_float(raw[j][w].y);
-                            v0[4 * w + 2] = __uint_as_float(raw[j][w].z);
-                            v0[4 * w + 3] = __uint_as_float(raw[j][w].w);
-                            v1[4 * w] = __uint_as_float(raw[j][4 + w].x);
-                            v1[4 * w + 1] = __uint_as_float(raw[j][4 + w].y);
-                            v1[4 * w + 2] = __uint_as_float(raw[j][4 + w].z);
-                            v1[4 * w + 3] = __uint_as_float(raw[j][4 + w].w);
+                        for (int w = 0; w < 8; ++w) {
+                            const bool lv = (w < words / 2) ? l0[j] : l1[j];
+                            raw[j][w] = (w < words && lv) ? __ldg(src + w) : make_uint4(0, 0, 0, 0);
                         }
-                    } else {
-                        unpack_bf16x8(raw[j][0], v0);
-                        unpack_bf16x8(raw[j][1], v0 + 8);
-                        unpack_bf16x8(raw[j][2], v1);
-                        unpack_bf16x8(raw[j][3], v1 + 8);
                     }
-                    uint32_t sb0, sb1;
-                    uint2 q0, q1;
-                    quantize_block16(v0, s_ga, l0[j], sb0, q0);
-                    quantize_block16(v1, s_ga, l1[j], sb1, q1);
-                    // K-major 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
-                    *reinterpret_cast<uint4*>(adst + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-                        make_uint4(q0.x, q0.y, q1.x, q1.y);
-                    // scale atom of k-step c / 2: row r at (r % 32) * 16 + (r / 32 % 4) * 4, block (c % 2) * 2
-                    *reinterpret_cast<uint16_t*>(sdst + (c >> 1) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
-                                                 (c & 1) * 2) = (uint16_t)(sb0 | (sb1 << 8));
+                    if (!waited) {
+                        if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
+                            ok = false;
+                            break;
+                        }
+                        waited = true;
+                    }
+#pragma unroll
+                    for (int j = 0; j < CB; ++j) {
+                        const int it = qt + 64 * (b0 + j);
+                        const int r = it >> 3, c = it & 7;
+                        float v0[16], v1[16];
+                        if (p.a_fp32) {
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) {
+                                v0[4 * w] = __uint_as_float(raw[j][w].x);
+                                v0[4 * w + 1] = __uint_as_float(raw[j][w].y);
+                                v0[4 * w + 2] = __uint_as_float(raw[j][w].z);
+                                v0[4 * w + 3] = __uint_as_float(raw[j][w].w);
+                                v1[4 * w] = __uint_as_float(raw[j][4 + w].x);
+                                v1[4 * w + 1] = __uint_as_float(raw[j][4 + w].y);
+                                v1[4 * w + 2] = __uint_as_float(raw[j][4 + w].z);
+                                v1[4 * w + 3] = __uint_as_float(raw[j][4 + w].w);
+                            }
+                        } else {
+                            unpack_bf16x8(raw[j][0], v0);
+                            unpack_bf16x8(raw[j][1], v0 + 8);
+                            unpack_bf16x8(raw[j][2], v1);
+                            unpack_bf16x8(raw[j][3], v1 + 8);
+                        }
+                        uint32_t sb0, sb1;
+                        uint2 q0, q1;
+                        quantize_block16(v0, s_ga, l0[j], sb0, q0);
+                        quantize_block16(v1, s_ga, l1[j], sb1, q1);
+                        // K-major 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+                        *reinterpret_cast<uint4*>(adst + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+                            make_uint4(q0.x, q0.y, q1.x, q1.y);
+                        // scale atom of k-step c / 2: row r at (r % 32) * 16 + (r / 32 % 4) * 4, block (c % 2) * 2
+                        *reinterpret_cast<uint16_t*>(sdst + (c >> 1) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
+                                                     (c & 1) * 2) = (uint16_t)(sb0 | (sb1 << 8));
+                    }
                 }
             }
-            if (!ok) break;
+            if (!ok) {
+                *bad = 1;
+                break;
+            }
             fence_proxy_async_shared();     // the MMA reads the stage through the async proxy
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[stage]);
@@ -379,45 +535,46 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                 stage = 0;
                 phase ^= 1;
             }
-            if (++kt == k_tiles) kt = 0;
+            u += st.nkt;
         }
     } else if (warp >= 8) {
         // ------------------------------------------------------------ scale staging
+        // Lane l of quadrant q writes TMEM lane 32q + l: row l of every atom
+        // (16 bytes = the scales of rows l, l+32, l+64, l+96), the layout the
+        // block-scaled MMA reads for both operands; each k-tile of the stage
+        // fills 16 columns of the slot's A half and 16 of its B half.
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         int stage = 0, slot = 0;
         uint32_t phase = 0, slot_phase = 0;
-        for (int64_t u = u_begin; u < u_end; ++u) {
+        for (int64_t u = u_begin; u < u_end;) {
+            const Stage st = stage_at(u, u_begin, u_end, k_tiles);
             if (!mbar_wait(&full[stage], phase, kStatusTimeoutFull) ||
-                !mbar_wait(&sf_free[slot], slot_phase ^ 1, kStatusTimeoutFull))
+                !mbar_wait(&sf_free[slot], slot_phase ^ 1, kStatusTimeoutFull)) {
+                *bad = 1;
                 break;
-            tc_fence_after();
-            const uint8_t* sfa = smem + OFF_SFA + stage * SFA_STAGE + lane * 16;
-            const uint8_t* sfb = smem + OFF_SFB + stage * SFB_STAGE + lane * 16;
-            uint32_t ra[16], rb[16], rc[16];
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint4 a = *reinterpret_cast<const uint4*>(sfa + ks * 512);
-                ra[4 * ks] = a.x;
-                ra[4 * ks + 1] = a.y;
-                ra[4 * ks + 2] = a.z;
-                ra[4 * ks + 3] = a.w;
-                const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + ks * 512);
-                const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + ks * 512);
-                uint32_t* d = ks < 2 ? rb : rc;
-                const int o = (ks & 1) * 8;
-                d[o] = b0.x;
-                d[o + 1] = b0.y;
-                d[o + 2] = b0.z;
-                d[o + 3] = b0.w;
-                d[o + 4] = b1.x;
-                d[o + 5] = b1.y;
-                d[o + 6] = b1.z;
-                d[o + 7] = b1.w;
             }
+            tc_fence_after();
             const uint32_t col = tmem_base + lane_base + SF_COL + slot * SF_SLOT;
-            tmem_st_32x32b_x16(col, ra);
-            tmem_st_32x32b_x16(col + 16, rb);
-            tmem_st_32x32b_x16(col + 32, rc);
+            for (int h = 0; h < st.nkt; ++h) {
+                const uint8_t* sfa = smem + OFF_SFA + stage * SF_STAGE + h * SF_KT + lane * 16;
+                const uint8_t* sfb = smem + OFF_SFB + stage * SF_STAGE + h * SF_KT + lane * 16;
+                uint32_t ra[16], rb[16];
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(sfa + ks * 512);
+                    const uint4 b = *reinterpret_cast<const uint4*>(sfb + ks * 512);
+                    ra[4 * ks] = a.x;
+                    ra[4 * ks + 1] = a.y;
+                    ra[4 * ks + 2] = a.z;
+                    ra[4 * ks + 3] = a.w;
+                    rb[4 * ks] = b.x;
+                    rb[4 * ks + 1] = b.y;
+                    rb[4 * ks + 2] = b.z;
+                    rb[4 * ks + 3] = b.w;
+                }
+                tmem_st_32x32b_x16(col + 16 * h, ra);        // A: k-step ks at columns 4 ks .. 4 ks + 3
+                tmem_st_32x32b_x16(col + 32 + 16 * h, rb);   // B: k-step ks at columns 32 + 4 ks ..
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -430,108 +587,90 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
                 slot = 0;
                 slot_phase ^= 1;
             }
+            u += st.nkt;
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
         // Per segment (one tile's k-range): the warps whose TMEM lanes hold
         // token rows move the FP32 accumulator into shared memory and release
-        // TMEM at once, so the MMAs of the next segment start while this one is
-        // stored.  Then all 128 epilogue threads work on the staged tile, 4
+        // it.  Then all 128 epilogue threads work on the staged tile, 4
         // consecutive columns of one row each: a contributor (a range that
-        // starts inside the tile) writes its partial to the workspace and
-        // publishes it; the owner of a tile that lies wholly in this range
-        // scales each column by s_ga * s_gw[seg] and stores the output.  An
-        // owner whose range ends inside the tile waits for the peers' flags and
-        // hands over to the all-warp finish below.  Every branch is uniform over
-        // the four warps, so the named barrier (id 1, 128 threads) always matches.
+        // starts inside the tile) writes its tagged partial to the workspace;
+        // the owner of a tile that lies wholly in this range scales each
+        // column by s_ga * s_gw[seg] and stores the output.  An owner whose
+        // range ends inside the tile hands over to the all-warp finish below.
+        // Every branch is uniform over the four warps, so the named barrier
+        // (id 1, 128 threads) always matches.
         const int quad = warp & 3;
         const int et = threadIdx.x - 128;          // 0..127
         const int t = quad * 32 + lane;            // token row = accumulator lane
         const bool live = quad * 32 < BT;          // warp holds loaded token rows
-        unsigned long long* flags = reinterpret_cast<unsigned long long*>(p.ws);
-        float* parts = reinterpret_cast<float*>(p.ws + FLAGS_BYTES);
         float s_ga = FQ ? 0.0f : *p.act_scale;        // FQ: known once the first stage is in
         const int units4 = min(p.m, BT) * (BN / 4);  // float4 units of the live rows
-        uint32_t segs = 0;
+        int seg = 0;
         int64_t u = u_begin;
         while (u < u_end) {
             const int nb = (int)(u / k_tiles), kb = (int)(u - (int64_t)nb * k_tiles);
             const int64_t seg_end = min(u_end, (int64_t)(nb + 1) * k_tiles);
             const bool owner = kb == 0;
             const bool complete = owner && seg_end == (int64_t)(nb + 1) * k_tiles;
-            const int last = owner && !complete ? cta_of_unit((int64_t)(nb + 1) * k_tiles - 1, p.units, p.ctas) : cta;
+            const int b = seg & 1;
 
-            if (et == 0) *acc_ok = mbar_wait(acc_full, segs & 1, kStatusTimeoutAccum) ? 1 : 0;
+            if (et == 0) *verdict = mbar_wait(&acc_full[b], (seg >> 1) & 1, kStatusTimeoutAccum) ? 1 : 0;
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (!*acc_ok) break;
-            if (FQ && segs == 0) {
+            if (!*verdict) {
+                if (et == 0) *bad = 1;
+                break;
+            }
+            if (FQ && seg == 0) {
                 // bounded like every wait; the quantiser set it before its first stage
-                if (et == 0) *sga_ok = mbar_wait(sga_ready, 0, kStatusTimeoutAccum) ? 1 : 0;
+                if (et == 0) *verdict = mbar_wait(sga_ready, 0, kStatusTimeoutAccum) ? 1 : 0;
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (!*sga_ok) break;
+                if (!*verdict) {
+                    if (et == 0) *bad = 1;
+                    break;
+                }
                 s_ga = *s_ga_smem;
             } else if (FQ) {
                 s_ga = *s_ga_smem;
             }
             tc_fence_after();
             if (live) {
-                const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16);
+                const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + b * BN;
                 float* row = acc_stage + t * ACC_PITCH;
-#pragma unroll 1
-                for (int j = 0; j < BN / 32; j += 2) {
-                    uint32_t r0[32], r1[32];
-                    __syncwarp();
-                    tmem_ld_32x32b_x32(taddr + j * 32, r0);
-                    tmem_ld_32x32b_x32(taddr + (j + 1) * 32, r1);
-                    tmem_ld_wait();
-                    if (t < BT) {
+                uint32_t r0[64], r1[64];
+                __syncwarp();
+                tmem_ld_32x32b_x64(taddr, r0);
+                tmem_ld_32x32b_x64(taddr + 64, r1);
+                tmem_ld_wait();
+                if (t < BT) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
-                            *reinterpret_cast<float4*>(row + j * 32 + e) =
-                                make_float4(__uint_as_float(r0[e]), __uint_as_float(r0[e + 1]),
-                                            __uint_as_float(r0[e + 2]), __uint_as_float(r0[e + 3]));
-                            *reinterpret_cast<float4*>(row + (j + 1) * 32 + e) =
-                                make_float4(__uint_as_float(r1[e]), __uint_as_float(r1[e + 1]),
-                                            __uint_as_float(r1[e + 2]), __uint_as_float(r1[e + 3]));
-                        }
+                    for (int e = 0; e < 64; e += 4) {
+                        *reinterpret_cast<float4*>(row + e) =
+                            make_float4(__uint_as_float(r0[e]), __uint_as_float(r0[e + 1]),
+                                        __uint_as_float(r0[e + 2]), __uint_as_float(r0[e + 3]));
+                        *reinterpret_cast<float4*>(row + 64 + e) =
+                            make_float4(__uint_as_float(r1[e]), __uint_as_float(r1[e + 1]),
+                                        __uint_as_float(r1[e + 2]), __uint_as_float(r1[e + 3]));
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-            ++segs;
-
-            if (owner && !complete) {
-                // thread i waits for CTAs cta + 1 + i, cta + 1 + i + 128, ... to
-                // publish their partials of tile nb
-                for (int i = et; i < last - cta; i += 128) {
-                    const long long t0 = clock64();
-                    while (ld_acquire_u64(flags + cta + 1 + i) != p.epoch) {
-                        if (clock64() - t0 > kWaitCycles) {
-                            record_status(kStatusTimeoutCluster);
-                            *peers_bad = 1;
-                            break;
-                        }
-                    }
-                }
-            }
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
+            ++seg;
             // An owner whose range ends inside tile nb (always the CTA's last
             // segment) leaves the reduction to all twelve warps, below.
             if (owner && !complete) break;
             asm volatile("bar.sync 1, 128;" ::: "memory");   // staged tile complete
-            if (*peers_bad) break;
 
             if (!owner) {
-                float* mine = parts + (int64_t)cta * BT * BN;
+                unsigned long long* mine = parts + (int64_t)cta * BT * BN;
                 for (int x = et; x < units4; x += 128) {
                     const int r = x / (BN / 4), c4 = x % (BN / 4);
-                    __stcg(reinterpret_cast<float4*>(mine + r * BN) + c4,
-                           *reinterpret_cast<const float4*>(acc_stage + r * ACC_PITCH + 4 * c4));
+                    st_tagged4(mine + r * BN + 4 * c4, *reinterpret_cast<const float4*>(acc_stage + r * ACC_PITCH + 4 * c4),
+                               tag);
                 }
-                __threadfence();
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (et == 0) st_release_u64(flags + cta, p.epoch);
             } else {
                 // a complete tile: scale and store
                 for (int x = et; x < units4; x += 128) {
@@ -549,55 +688,78 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
     // ---------------------------------------------------------------- split-tile finish
     // The CTA whose range starts tile nb = (u_end - 1) / k_tiles but ends inside
     // it owns that tile's result: once the epilogue has staged this CTA's
-    // accumulator and acquired the peers' flags, all 384 threads add the peers'
-    // FP32 partials in CTA order (loads for FPG peers in flight together),
-    // scale and store.  The condition is the same for every thread.
+    // accumulator, all 384 threads add the contributors' partials (CTAs
+    // cta + 1 .. last, in that order; FPG of them in flight per item and FDU
+    // items per thread, each word waited for until it carries this call's
+    // tag), scale and store.  The condition is the same for every thread.
     {
-        const int64_t fin_nb = u_end > u_begin ? (u_end - 1) / k_tiles : 0;
-        const bool finish = u_end > u_begin && u_end % k_tiles != 0 && fin_nb * k_tiles >= u_begin;
+        const int64_t fin_nb = (u_end - 1) / k_tiles;
+        const bool finish = u_end % k_tiles != 0 && fin_nb * k_tiles >= u_begin;
         if (finish) {
             asm volatile("bar.sync 2, 384;" ::: "memory");
-            if (*acc_ok && !*peers_bad) {
-                constexpr int FDU = 3, FPG = 8;
+            dependency_wait();
+            if (!*bad) {
+                constexpr int FDU = 2, FPG = 4;
                 const int nb = (int)fin_nb;
                 const int last = cta_of_unit((int64_t)(nb + 1) * k_tiles - 1, p.units, p.ctas);
                 const int units4 = min(p.m, BT) * (BN / 4);
-                const float* parts = reinterpret_cast<const float*>(p.ws + FLAGS_BYTES);
                 const float s_ga = FQ ? *s_ga_smem : *p.act_scale;
                 for (int x0 = threadIdx.x; x0 < units4; x0 += FDU * THREADS) {
                     float4 v[FDU];
+                    int64_t off[FDU];
 #pragma unroll
                     for (int i = 0; i < FDU; ++i) {
-                        const int x = x0 + i * THREADS;
-                        if (x < units4)
-                            v[i] = *reinterpret_cast<const float4*>(acc_stage + (x / (BN / 4)) * ACC_PITCH +
-                                                                    4 * (x % (BN / 4)));
+                        const int x = min(x0 + i * THREADS, units4 - 1);
+                        off[i] = (int64_t)(x / (BN / 4)) * BN + 4 * (x % (BN / 4));
+                        v[i] = *reinterpret_cast<const float4*>(acc_stage + (x / (BN / 4)) * ACC_PITCH +
+                                                                4 * (x % (BN / 4)));
                     }
                     for (int c2 = cta + 1; c2 <= last; c2 += FPG) {
-                        float4 q[FPG][FDU];
+                        Tagged4 q[FDU][FPG];
 #pragma unroll
-                        for (int g = 0; g < FPG; ++g) {
-                            const float* src = parts + (int64_t)(c2 + g) * BT * BN;
+                        for (int g = 0; g < FPG; ++g)
 #pragma unroll
-                            for (int i = 0; i < FDU; ++i) {
-                                const int x = x0 + i * THREADS;
-                                if (x < units4 && c2 + g <= last)
-                                    q[g][i] = __ldcg(reinterpret_cast<const float4*>(
-                                        src + (x / (BN / 4)) * BN + 4 * (x % (BN / 4))));
-                            }
-                        }
+                            for (int i = 0; i < FDU; ++i)
+                                if (c2 + g <= last) ld_tagged4(parts + (int64_t)(c2 + g) * BT * BN + off[i], q[i][g]);
+                        uint32_t pending = 0;
 #pragma unroll
-                        for (int g = 0; g < FPG; ++g) {
-                            if (c2 + g <= last) {
+                        for (int g = 0; g < FPG; ++g)
 #pragma unroll
-                                for (int i = 0; i < FDU; ++i) {
-                                    v[i].x = __fadd_rn(v[i].x, q[g][i].x);
-                                    v[i].y = __fadd_rn(v[i].y, q[g][i].y);
-                                    v[i].z = __fadd_rn(v[i].z, q[g][i].z);
-                                    v[i].w = __fadd_rn(v[i].w, q[g][i].w);
+                            for (int i = 0; i < FDU; ++i)
+                                if (c2 + g <= last && !tagged4_ok(q[i][g], tag)) pending |= 1u << (g * FDU + i);
+                        if (pending) {
+                            const long long t0 = clock64();
+                            while (pending) {
+#pragma unroll
+                                for (int g = 0; g < FPG; ++g)
+#pragma unroll
+                                    for (int i = 0; i < FDU; ++i)
+                                        if (pending & (1u << (g * FDU + i)))
+                                            ld_tagged4(parts + (int64_t)(c2 + g) * BT * BN + off[i], q[i][g]);
+#pragma unroll
+                                for (int g = 0; g < FPG; ++g)
+#pragma unroll
+                                    for (int i = 0; i < FDU; ++i)
+                                        if ((pending & (1u << (g * FDU + i))) && tagged4_ok(q[i][g], tag))
+                                            pending &= ~(1u << (g * FDU + i));
+                                if (pending && clock64() - t0 > kWaitCycles) {
+                                    record_status(kStatusTimeoutCluster);
+                                    *bad = 1;
+                                    break;
                                 }
                             }
                         }
+#pragma unroll
+                        for (int g = 0; g < FPG; ++g)
+#pragma unroll
+                            for (int i = 0; i < FDU; ++i)
+                                if (c2 + g <= last) {
+                                    const float4 w = tagged4_value(q[i][g]);
+                                    v[i].x = __fadd_rn(v[i].x, w.x);
+                                    v[i].y = __fadd_rn(v[i].y, w.y);
+                                    v[i].z = __fadd_rn(v[i].z, w.z);
+                                    v[i].w = __fadd_rn(v[i].w, w.w);
+                                }
                     }
 #pragma unroll
                     for (int i = 0; i < FDU; ++i) {

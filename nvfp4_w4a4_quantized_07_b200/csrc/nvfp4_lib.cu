@@ -131,6 +131,51 @@ nvfp4_status encode_fp4_map(CUtensorMap* map, const uint8_t* base, int64_t rows,
     return NVFP4_OK;
 }
 
+// 3-D view {128 bytes, rows, K / 256} of a packed FP4 buffer (row stride K/2
+// bytes, k-tile stride 128 bytes) for boxes of two k-tiles of box_rows rows,
+// which land as two consecutive 128-byte-swizzled tiles.  Needs K % 256 == 0,
+// so every box lies inside the buffer.
+nvfp4_status encode_fp4_map3(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t k, int box_rows)
+{
+    const cuuint64_t dims[3] = {128u, (cuuint64_t)rows, (cuuint64_t)(k / 256)};
+    const cuuint64_t strides[2] = {(cuuint64_t)(k / 2), 128u};
+    const cuuint32_t box[3] = {128u, (cuuint32_t)box_rows, 2u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+    return NVFP4_OK;
+}
+
+// The decode kernel's maps: A with boxes of bt rows, W with boxes of 128 rows,
+// and their two-k-tile 3-D views when K is a multiple of 256 (else copies of
+// the 2-D maps, which the kernel then never reads as 3-D).  a_q == nullptr:
+// the activations are quantised inside the kernel and A's maps are unused.
+nvfp4_status encode_decode_maps(DecodeMaps* m, const uint8_t* a_q, const uint8_t* w_q, int64_t rows_a, int64_t n,
+                                int64_t k, int bt)
+{
+    nvfp4_status st = encode_fp4_map(&m->w, w_q, n, k, decode::BN);
+    if (st != NVFP4_OK) return st;
+    if (a_q != nullptr) {
+        if ((st = encode_fp4_map(&m->a, a_q, rows_a, k, bt)) != NVFP4_OK) return st;
+    } else {
+        m->a = m->w;
+    }
+    if (k % 256 == 0) {
+        if ((st = encode_fp4_map3(&m->w3, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
+        if (a_q != nullptr) {
+            if ((st = encode_fp4_map3(&m->a3, a_q, rows_a, k, bt)) != NVFP4_OK) return st;
+        } else {
+            m->a3 = m->w3;
+        }
+    } else {
+        m->w3 = m->w;
+        m->a3 = m->a;
+    }
+    return NVFP4_OK;
+}
+
 // Output C (m x n, row stride ldc elements) for TMA stores of 32-column
 // chunks from swizzled shared memory: BF16 chunks are 16 rows of 64 bytes
 // (64-byte swizzle); the FP32 map (32 x 32, 128-byte swizzle) is encoded for
@@ -267,17 +312,18 @@ nvfp4_status check_segments(const nvfp4_segment* segs, int nsegs, int64_t n, Seg
     return NVFP4_OK;
 }
 
-// Bytes of workspace the decode kernel needs for m tokens: flags plus one FP32
-// partial tile per CTA.
+// Bytes of workspace the decode kernel needs for m tokens: one partial tile
+// (16, 32 or 64 rows x 128 columns of tagged 8-byte words) per CTA slot.
 size_t decode_ws_bytes(int64_t m)
 {
     const int64_t bt = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
-    return (size_t)decode::FLAGS_BYTES + (size_t)decode::MAX_CTAS * (size_t)bt * decode::BN * 4;
+    return (size_t)decode::MAX_CTAS * (size_t)bt * decode::BN * 8;
 }
 
-// Per-call flag values for the decode kernel's partial-tile hand-off: a random
-// 64-bit starting point (so values left in a reused workspace by another
-// process or an aborted call cannot match) advanced once per call.
+// Per-call tags for the decode kernel's partial-tile hand-off: a random
+// starting point (so words left in a reused workspace by another process or an
+// aborted call do not match) advanced once per call; the kernel uses the low
+// 32 bits, which repeat only after 2^31 calls.
 std::atomic<unsigned long long> g_epoch{0};
 std::once_flag g_epoch_once;
 
@@ -293,36 +339,38 @@ unsigned long long next_epoch()
 }
 
 template <int BT, bool FQ>
-nvfp4_status launch_decode(const CUtensorMap& ta, const CUtensorMap& tw, const GemmParams& p, cudaStream_t s)
+nvfp4_status launch_decode(const DecodeMaps& maps, const GemmParams& p, cudaStream_t s)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.ctas, 1, 1);
     cfg.blockDim = dim3(decode::THREADS, 1, 1);
     cfg.dynamicSmemBytes = decode::Cfg<BT>::SMEM_BYTES;
     cfg.stream = s;
-    // The owners of split row tiles wait for the other CTAs' partials, so all
-    // CTAs must be resident at once.
+    // Programmatic dependent launch: the CTAs may start while the previous
+    // kernel in the stream is still running; each touches only weights until
+    // it has waited for that kernel (griddepcontrol.wait).  The grid is at
+    // most one CTA per SM, so once the previous kernel is done every CTA is
+    // resident; the participants of split tiles wait for each other's
+    // partials with a bounded wait.
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT, FQ>, ta, tw, p));
+    NVFP4_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_decode_kernel<BT, FQ>, maps, p));
     return NVFP4_OK;
 }
 
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Built-in scratch of nvfp4_gemm_decode_noalloc: the decode kernel's flags and
-// partial tiles for up to NVFP4_NOALLOC_MAX_M tokens and 256 CTA slots, in
-// device memory reserved when the module is loaded on a device (no allocation
-// call).  Its address on each device is looked up once, with that device
-// current.
+// Built-in scratch of nvfp4_gemm_decode_noalloc: the decode kernel's partial
+// tiles for up to NVFP4_NOALLOC_MAX_M tokens and every CTA slot, in device
+// memory reserved when the module is loaded on a device (no allocation call).
+// Its address on each device is looked up once, with that device current.
 // ---------------------------------------------------------------------------
-static_assert(NVFP4_NOALLOC_SCRATCH_BYTES ==
-                  decode::FLAGS_BYTES + (size_t)decode::MAX_CTAS * NVFP4_NOALLOC_MAX_M * decode::BN * 4,
-              "scratch = flags + one 16-row partial tile per CTA slot");
+static_assert(NVFP4_NOALLOC_SCRATCH_BYTES == (size_t)decode::MAX_CTAS * NVFP4_NOALLOC_MAX_M * decode::BN * 8,
+              "scratch = one 16-row partial tile per CTA slot");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NVFP4_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -677,11 +725,11 @@ static nvfp4_status gemm_impl(const uint8_t* a_q, const uint8_t* a_sf, const flo
     p.epoch = next_epoch();
     p.m_tiles = 1;
     p.n_tiles = w_tiles;
-    if ((st = encode_fp4_map(&ta, a_q, m, k, bt)) != NVFP4_OK) return st;
-    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
-    if (bt == 16) st = launch_decode<16, false>(ta, tw, p, s);
-    else if (bt == 32) st = launch_decode<32, false>(ta, tw, p, s);
-    else st = launch_decode<64, false>(ta, tw, p, s);
+    DecodeMaps maps;
+    if ((st = encode_decode_maps(&maps, a_q, w_q, m, n, k, bt)) != NVFP4_OK) return st;
+    if (bt == 16) st = launch_decode<16, false>(maps, p, s);
+    else if (bt == 32) st = launch_decode<32, false>(maps, p, s);
+    else st = launch_decode<64, false>(maps, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
 }
@@ -835,12 +883,11 @@ nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int64_t m, in
     p.epoch = next_epoch();
     p.m_tiles = 1;
     p.n_tiles = w_tiles;
-    CUtensorMap tw;
-    if ((st = encode_fp4_map(&tw, w_q, n, k, decode::BN)) != NVFP4_OK) return st;
-    // the A map is not read when the quantisation is fused in
-    if (bt == 16) st = launch_decode<16, true>(tw, tw, p, s);
-    else if (bt == 32) st = launch_decode<32, true>(tw, tw, p, s);
-    else st = launch_decode<64, true>(tw, tw, p, s);
+    DecodeMaps maps;   // the A maps are not read when the quantisation is fused in
+    if ((st = encode_decode_maps(&maps, nullptr, w_q, m, n, k, bt)) != NVFP4_OK) return st;
+    if (bt == 16) st = launch_decode<16, true>(maps, p, s);
+    else if (bt == 32) st = launch_decode<32, true>(maps, p, s);
+    else st = launch_decode<64, true>(maps, p, s);
     if (st != NVFP4_OK) return st;
     return ok();
 }

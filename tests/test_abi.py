@@ -179,7 +179,7 @@ def test_decode_noalloc_limits_without_a_device(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 64, 64, s, 1, FAKE, 0, 64, None) == 0
     assert nv.NVFP4_NOALLOC_MAX_M == 16
     # the built-in scratch is exactly the decode workspace for 16 tokens
-    assert lib.nvfp4_gemm_workspace_size(16, 64, 64, nv.NVFP4_GEMM_FORCE_DECODE) == 2048 + 256 * 16 * 256 * 4
+    assert lib.nvfp4_gemm_workspace_size(16, 64, 64, nv.NVFP4_GEMM_FORCE_DECODE) == 160 * 16 * 128 * 8
 
 
 def test_silu_mul_quantize_argument_errors(lib):
