@@ -444,72 +444,18 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
         out["gdn_gate_epilogue"] = {"heads": heads, "gemm_ms": ms_plain, "gemm_gdn_ms": ms_gdn,
                                     "overhead_pct": 100.0 * (ms_gdn / ms_plain - 1.0)}
 
-    # ---- calibrated FP8 KV cache: one layer's new K/V rows quantised and
-    # scattered into shuffled cache slots (prefill and decode sizes)
-    kv = {}
-    for tokens in (8192, 16):
-        k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens))
-        ks = torch.empty(1, dtype=torch.float32, device=device)
-        vs = torch.empty(1, dtype=torch.float32, device=device)
-        nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
-        nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
-        gen = torch.Generator().manual_seed(tokens)
-        slots = torch.randperm(2 * tokens, generator=gen)[:tokens].to(torch.int64).to(device)
-        kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
-        vc = torch.empty_like(kc)
-        ms = _timed(lambda: nv.kv_cache_quantize_fp8(k_rows, v_rows, ks, vs, kc, vc, slots), flush, stream, device)
-        nbytes = 2 * k_rows.numel() * (k_rows.element_size() + 1) + slots.numel() * 8
-        kv[f"tokens{tokens}_width{k_rows.shape[1]}"] = {
-            "us": ms * 1e3, "GB/s": nbytes / (ms * 1e-3) / 1e9, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-    out["kv_cache_fp8"] = {"bytes": "K and V in (bf16) + cache bytes out + int64 slot table", "shapes": kv}
-
-    # ---- decode sweep: HBM GB/s of the small-M GEMM (L2 flushed before each launch)
+    # ---- calibrated FP8 KV cache (one layer's new K/V rows quantised and
+    # scattered into shuffled cache slots) and the decode sweep (config 5):
+    # short kernels, timed back to back over inputs larger than twice the L2
+    kv, w1 = kv_back_to_back(nv, synthetic, device, stream, peaks)
+    out["kv_cache_fp8"] = {"bytes": "K and V in (bf16) + cache bytes out + int64 slot table",
+                           "timing": "60 launches back to back, median of 3", "shapes": kv}
     if not args.no_decode:
-        dec = {}
-        for shape in synthetic.DECODE_SHAPES:
-            widths, k, stds = synthetic.DECODE_SHAPES[shape]
-            mods = [synthetic.weights(n_i, k, s_i, seed=1 + i).to(device) for i, (n_i, s_i) in
-                    enumerate(zip(widths, stds))]
-            fwd = nv.quantize_weight(mods)
-            del mods
-            for m in synthetic.DECODE_M:
-                a, _ = synthetic.activations(m, k, seed=0, n_outliers=0)
-                a = a.to(device)
-                aqd = nv.quantize_act(a, act_scale=act_scale)
-                cd = torch.empty((m, fwd.n), dtype=torch.bfloat16, device=device)
-                times = []
-                for it in range(13):
-                    flush.zero_()
-                    torch.cuda._sleep(400_000)       # keep host launch latency out of the events
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    nv.gemm(aqd, fwd, out=cd)
-                    e1.record(stream)
-                    torch.cuda.synchronize(device)
-                    if it >= 3:
-                        times.append(e0.elapsed_time(e1))
-                ms = statistics.median(times)
-                nbytes = fwd.n * k // 2 + fwd.n * k // 16 + m * k // 2 + m * k // 16 + m * fwd.n * 2
-                gbs = nbytes / (ms * 1e-3) / 1e9
-                # the whole layer in one launch: quantisation fused into the decode GEMM
-                ltimes = []
-                for it in range(13):
-                    flush.zero_()
-                    torch.cuda._sleep(400_000)
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    nv.linear_decode(a, fwd, act_scale=act_scale, out=cd)
-                    e1.record(stream)
-                    torch.cuda.synchronize(device)
-                    if it >= 3:
-                        ltimes.append(e0.elapsed_time(e1))
-                lms = statistics.median(ltimes)
-                lbytes = fwd.n * k // 2 + fwd.n * k // 16 + m * k * 2 + m * fwd.n * 2
-                dec[f"m{m}_{shape}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
-                                        "frac_8TBs": gbs / 8000.0, "layer_us": lms * 1e3,
-                                        "layer_GB/s": lbytes / (lms * 1e-3) / 1e9}
-            del fwd
-        out["decode"] = {"unit": "GB/s", "bytes": "W_q + W_sf + A_q + A_sf + C (bf16), L2 flushed",
+        dec, w2 = decode_back_to_back(nv, synthetic, act_scale, device, stream, peaks)
+        out["decode"] = {"unit": "GB/s", "bytes": "W_q + W_sf + A_q + A_sf + C (bf16)",
+                         "timing": "60 launches back to back (programmatic dependent launch), weights rotated "
+                                   "over copies > 2x L2, median of 3",
+                         "max_enqueue_over_sleep": max(w1, w2),
                          "layer": "nvfp4_linear_decode: bf16 A quantised inside the GEMM, static scale; "
                                   "bytes W_q + W_sf + A (bf16) + C (bf16)",
                          "shapes": dec}
@@ -763,33 +709,119 @@ def run_decode_case(args):
 
 
 def _back_to_back_us(launches, stream, device, reps=3):
-    """Per-launch device time (us) of ``launches`` run back to back: a GPU sleep
-    of ~10 ms (longer than the host needs to enqueue them) precedes the first,
-    so the events see only the kernels and the gaps between them.  Median of
-    ``reps``."""
+    """Per-launch device time (us) of ``launches`` run back to back, median of
+    ``reps`` runs.  A GPU sleep precedes the first launch so that the host
+    enqueues all of them while the GPU waits; the host's enqueue time is
+    measured against the sleep's device duration, and a run whose enqueueing
+    took more than half of the sleep is repeated with a sleep twice as long,
+    so no host gap enters the event span.  Returns (us per launch, the largest
+    enqueue / sleep ratio among the kept runs)."""
+    import time
+
     import torch
     for f in launches[:4]:
         f()
     torch.cuda.synchronize(device)
-    res = []
-    for _ in range(reps):
-        torch.cuda._sleep(20_000_000)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cycles = 20_000_000
+    res, worst = [], 0.0
+    while len(res) < reps:
+        es, e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        es.record(stream)
+        torch.cuda._sleep(cycles)
         e0.record(stream)
+        t0 = time.perf_counter()
         for f in launches:
             f()
+        enqueue_ms = (time.perf_counter() - t0) * 1e3
         e1.record(stream)
         torch.cuda.synchronize(device)
+        ratio = enqueue_ms / max(es.elapsed_time(e0), 1e-3)
+        if ratio > 0.5:
+            if cycles >= 1 << 30:
+                raise RuntimeError(f"host enqueue ({enqueue_ms:.2f} ms) outlasts the GPU sleep")
+            cycles *= 2
+            continue
+        worst = max(worst, ratio)
         res.append(e0.elapsed_time(e1) * 1e3 / len(launches))
-    return statistics.median(res)
+    return statistics.median(res), worst
+
+
+def decode_back_to_back(nv, synthetic, act_scale, device, stream, peaks, ms=None, shapes=None, layer=True):
+    """Decode GEMMs (config 5) timed as 60 launches back to back, each on one of
+    several copies of the fused weight that together exceed twice the L2, so
+    every launch streams its weight from HBM while the next one's start
+    overlaps its tail (the kernel's programmatic dependent launch).  GB/s of
+    the algorithmic bytes W_q + W_sf + A_q + A_sf + C (BF16) per (m, shape),
+    and the same for the whole layer in one launch (nvfp4_linear_decode:
+    bytes W_q + W_sf + BF16 A + C)."""
+    import dataclasses
+
+    import torch
+    l2_twice = 2 * 126 * 1024 * 1024
+    ms = synthetic.DECODE_M if ms is None else ms
+    out, worst = {}, 0.0
+    for shape in (synthetic.DECODE_SHAPES if shapes is None else shapes):
+        widths, k, stds = synthetic.DECODE_SHAPES[shape]
+        mods = [synthetic.weights(n_i, k, s_i, seed=1 + i).to(device) for i, (n_i, s_i) in
+                enumerate(zip(widths, stds))]
+        fw = nv.quantize_weight(mods)
+        del mods
+        wbytes = fw.q.numel() + fw.sf.numel()
+        copies = [fw] + [dataclasses.replace(fw, q=fw.q.clone(), sf=fw.sf.clone())
+                         for _ in range(max(1, -(-l2_twice // wbytes)) - 1)]
+        for m in ms:
+            a, _ = synthetic.activations(m, k, seed=0, n_outliers=0)
+            a = a.to(device)
+            aq = nv.quantize_act(a, act_scale=act_scale)
+            c = torch.empty((m, fw.n), dtype=torch.bfloat16, device=device)
+            launches = [(lambda w=copies[i % len(copies)]: nv.gemm(aq, w, out=c)) for i in range(60)]
+            us, r = _back_to_back_us(launches, stream, device)
+            worst = max(worst, r)
+            nbytes = wbytes + aq.q.numel() + m * k // 16 + c.numel() * 2
+            gbs = nbytes / (us * 1e-6) / 1e9
+            row = {"us": us, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "frac_8TBs": gbs / 8000.0}
+            if layer:
+                lays = [(lambda w=copies[i % len(copies)]: nv.linear_decode(a, w, act_scale=act_scale, out=c))
+                        for i in range(60)]
+                lus, r = _back_to_back_us(lays, stream, device)
+                worst = max(worst, r)
+                lbytes = wbytes + a.numel() * 2 + c.numel() * 2
+                row.update({"layer_us": lus, "layer_GB/s": lbytes / (lus * 1e-6) / 1e9})
+            out[f"m{m}_{shape}"] = row
+        del copies, fw
+    return out, worst
+
+
+def kv_back_to_back(nv, synthetic, device, stream, peaks, tokens=8192):
+    """The FP8 KV-cache kernel (one layer's K and V rows quantised and scattered
+    into shuffled cache slots) as 60 launches back to back over input sets that
+    together exceed twice the L2."""
+    import torch
+    l2_twice = 2 * 126 * 1024 * 1024
+    probe = synthetic.kv_rows(tokens, seed=11)
+    per_set = 2 * probe[0].numel() * (probe[0].element_size() + 1) + tokens * 8
+    sets = []
+    for r in range(max(2, -(-l2_twice // per_set))):
+        k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens, seed=11 + r))
+        ks = torch.empty(1, dtype=torch.float32, device=device)
+        vs = torch.empty(1, dtype=torch.float32, device=device)
+        nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
+        nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
+        slots = torch.randperm(2 * tokens, generator=torch.Generator().manual_seed(r))[:tokens].to(device)
+        kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
+        sets.append((k_rows, v_rows, ks, vs, kc, torch.empty_like(kc), slots))
+    launches = [(lambda s_=sets[i % len(sets)]: nv.kv_cache_quantize_fp8(*s_)) for i in range(60)]
+    us, worst = _back_to_back_us(launches, stream, device)
+    gbs = per_set / (us * 1e-6) / 1e9
+    return {f"tokens{tokens}_width{probe[0].shape[1]}": {
+        "us": us, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"], "input_sets": len(sets),
+        "bytes_rotated": per_set * len(sets)}}, worst
 
 
 def run_short_kernels(args):
-    """Decode GEMMs (m = 16) and the FP8 KV-cache kernel timed as 60 launches
-    back to back, each on one of several input copies that together exceed
-    twice the L2, so every launch streams its operands from HBM."""
-    import dataclasses
-
+    """The decode GEMMs (m = 16) and the FP8 KV-cache kernel timed back to back
+    (see decode_back_to_back and kv_back_to_back), without the rest of the
+    bench."""
     import torch
 
     import nvfp4_w4a4_quantized_07_b200 as nv
@@ -801,45 +833,11 @@ def run_short_kernels(args):
     device = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(device)
     peaks, _ = measured_peaks()
-    l2_twice = 2 * 126 * 1024 * 1024
+    dec, w1 = decode_back_to_back(nv, synthetic, None, device, stream, peaks, ms=[16], layer=False)
+    kv, w2 = kv_back_to_back(nv, synthetic, device, stream, peaks)
     out = {"method": "60 launches back to back behind a GPU sleep, inputs rotated over copies > 2x L2; "
-                     "median of 3 runs", "decode_m16": {}, "kv_cache_fp8": {}}
-    for shape, (widths, k, stds) in synthetic.DECODE_SHAPES.items():
-        mods = [synthetic.weights(n_i, k, s_i, seed=1 + i).to(device) for i, (n_i, s_i) in
-                enumerate(zip(widths, stds))]
-        fw = nv.quantize_weight(mods)
-        del mods
-        wbytes = fw.q.numel() + fw.sf.numel()
-        copies = [fw] + [dataclasses.replace(fw, q=fw.q.clone(), sf=fw.sf.clone())
-                         for _ in range(max(1, -(-l2_twice // wbytes)) - 1)]
-        a, _ = synthetic.activations(16, k, seed=0, n_outliers=0)
-        aq = nv.quantize_act(a.to(device))
-        c = torch.empty((16, fw.n), dtype=torch.bfloat16, device=device)
-        launches = [(lambda w=copies[i % len(copies)]: nv.gemm(aq, w, out=c)) for i in range(60)]
-        us = _back_to_back_us(launches, stream, device)
-        nbytes = wbytes + aq.q.numel() + aq.sf.numel() + c.numel() * 2
-        out["decode_m16"][shape] = {"us": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
-                                    "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                                    "weight_copies": len(copies)}
-        del copies, fw
-    tokens = 8192
-    sets = []
-    for r in range(6):
-        k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens, seed=11 + r))
-        ks = torch.empty(1, dtype=torch.float32, device=device)
-        vs = torch.empty(1, dtype=torch.float32, device=device)
-        nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
-        nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
-        slots = torch.randperm(2 * tokens, generator=torch.Generator().manual_seed(r))[:tokens].to(device)
-        kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
-        sets.append((k_rows, v_rows, ks, vs, kc, torch.empty_like(kc), slots))
-    launches = [(lambda s_=sets[i % len(sets)]: nv.kv_cache_quantize_fp8(*s_)) for i in range(60)]
-    us = _back_to_back_us(launches, stream, device)
-    k0 = sets[0][0]
-    nbytes = 2 * k0.numel() * (k0.element_size() + 1) + tokens * 8
-    out["kv_cache_fp8"][f"tokens{tokens}_width{k0.shape[1]}"] = {
-        "us": us, "GB/s": nbytes / (us * 1e-6) / 1e9, "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-        "input_copies": len(sets)}
+                     "median of 3 runs", "max_enqueue_over_sleep": max(w1, w2),
+           "decode_m16": {k.split("_", 1)[1]: v for k, v in dec.items()}, "kv_cache_fp8": kv}
     print(json.dumps(out), flush=True)
     return 0
 

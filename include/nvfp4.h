@@ -393,7 +393,10 @@ NVFP4_API nvfp4_status nvfp4_fp8_calibrate(const void* x, nvfp4_in_dtype dt, int
  *   slot_mapping      device int64[tokens]: the cache row of each token; a
  *                     negative entry (padding) or one >= num_slots is
  *                     skipped.  NULL: token t goes to slot t (then tokens <=
- *                     num_slots).
+ *                     num_slots).  The valid entries must be distinct: each
+ *                     16-element piece of a row is written on its own, so two
+ *                     tokens mapped to one slot leave that row a mix of both
+ *                     (which pieces come from which token is unspecified).
  *   k_scale_dev,
  *   v_scale_dev       device floats, the calibrated scales.
  *   k_cache, v_cache  device, num_slots rows of width bytes, row stride

@@ -143,9 +143,22 @@ def sf_offset(row: int, kblock: int, k: int) -> int:
     return int(load().nvfp4_sf_offset(row, kblock, k))
 
 
+_quant_ws_cache = {}
+
+
 def quant_workspace(device) -> "torch.Tensor":
+    """A cached per-device workspace of nvfp4_quant_workspace_size bytes for the
+    dynamic-scale quantisers.  It needs no initialisation (the library clears
+    the amax word it uses on the call's stream), so it is allocated once per
+    device and not filled; calls that may run concurrently on different
+    streams must pass workspaces of their own."""
     import torch
-    return torch.zeros(load().nvfp4_quant_workspace_size(), dtype=torch.uint8, device=device)
+    key = torch.device(device)
+    ws = _quant_ws_cache.get(key)
+    if ws is None:
+        ws = torch.empty(load().nvfp4_quant_workspace_size(), dtype=torch.uint8, device=key)
+        _quant_ws_cache[key] = ws
+    return ws
 
 
 @dataclass
@@ -273,7 +286,8 @@ _ws_cache = {}
 
 
 def gemm_workspace(m: int, n: int, k: int, flags: int, device):
-    """A cached per-device workspace of at least nvfp4_gemm_workspace_size bytes."""
+    """A cached per-device workspace of at least nvfp4_gemm_workspace_size bytes
+    (it needs no initialisation: the decode kernel tags what it writes)."""
     import torch
     need = int(load().nvfp4_gemm_workspace_size(m, n, k, flags))
     if need == 0:
@@ -281,7 +295,7 @@ def gemm_workspace(m: int, n: int, k: int, flags: int, device):
     key = torch.device(device)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
-        ws = torch.zeros(need, dtype=torch.uint8, device=key)
+        ws = torch.empty(need, dtype=torch.uint8, device=key)
         _ws_cache[key] = ws
     return ws
 

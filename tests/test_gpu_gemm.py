@@ -197,20 +197,56 @@ def test_config_prefill_4096x5120x5120_sampled_rows():
     assert torch.equal(c.cpu(), c32.cpu().to(torch.bfloat16))
 
 
-def test_config_fused_gdn_in_proj_8192_sampled_rows():
+@pytest.mark.parametrize("flags", [AUTO, PAIR])
+def test_config_fused_gdn_in_proj_8192_sampled_rows(flags):
     """8192 x 5120 activations against six separately calibrated modules
-    [2048, 2048, 4096, 4096, 48, 48] (N = 12384), checked against the six
-    unfused GEMMs too."""
+    [2048, 2048, 4096, 4096, 48, 48] (N = 12384), checked against the oracle
+    and the six unfused GEMMs on sampled rows; one shared global scale
+    (module 0's, or the largest) must fail the same check at this size."""
     p = synthetic.gdn_in_proj()
-    c32, aq, fw = _run_linear(p, AUTO, torch.float32)
+    c32, aq, fw = _run_linear(p, flags, torch.float32)
     rows = _sample_rows(p.m, 32)
     c64, a_hat, w_hat = _oracle_linear(p, rows=rows)
     rsel = torch.from_numpy(rows).cuda()
     assert_gemm_close(c32[rsel], c64, a_hat, w_hat, "gdn in-proj")
+    parts = [nv.gemm(aq, nv.quantize_weight([w.cuda()]), out_dtype=torch.float32, flags=flags)[rsel]
+             for w in p.modules]
+    torch.cuda.synchronize()
+    unfused = torch.cat(parts, dim=1)
+    assert_gemm_close(c32[rsel], unfused.double().cpu().numpy(), a_hat, w_hat, "fused vs unfused")
+    scales = [s for _, _, s in fw.segments]
+    for shared in (scales[0], max(scales)):
+        bad = nv.gemm(aq, fw, out_dtype=torch.float32, flags=flags, segments=[(0, fw.n, shared)])[rsel]
+        torch.cuda.synchronize()
+        ratio, fro = gemm_check(bad, c64, a_hat, w_hat)
+        assert ratio > 1.0 and fro > 2e-3, (shared, ratio, fro)
+
+
+def test_config_mlp_gate_up_fused_equals_unfused_and_shared_scale_fails():
+    """The long-prefill MLP's fused gate/up GEMM (32768 x 5120 against two
+    separately calibrated 17408-row modules, N = 34816) against the oracle and
+    its two unfused GEMMs on sampled rows; one shared global scale (either
+    module's) must fail the same check."""
+    p = synthetic.mlp_gate_up()
+    c32, aq, fw = _run_linear(p, AUTO, torch.float32)
+    rows = _sample_rows(p.m, 6)
+    c64, a_hat, w_hat = _oracle_linear(p, rows=rows)
+    rsel = torch.from_numpy(rows).cuda()
+    assert_gemm_close(c32[rsel], c64, a_hat, w_hat, "mlp gate/up")
     parts = [nv.gemm(aq, nv.quantize_weight([w.cuda()]), out_dtype=torch.float32)[rsel] for w in p.modules]
     torch.cuda.synchronize()
     unfused = torch.cat(parts, dim=1)
     assert_gemm_close(c32[rsel], unfused.double().cpu().numpy(), a_hat, w_hat, "fused vs unfused")
+    # Both modules are N(0, 0.02): their scales differ by only ~0.4 %, so a
+    # shared scale stays inside the per-element bound and fails on the
+    # Frobenius error alone (about 3e-3 against 2e-3).
+    scales = [s for _, _, s in fw.segments]
+    assert len(scales) == 2 and scales[0] != scales[1]
+    for shared in scales:
+        bad = nv.gemm(aq, fw, out_dtype=torch.float32, segments=[(0, fw.n, shared)])[rsel]
+        torch.cuda.synchronize()
+        ratio, fro = gemm_check(bad, c64, a_hat, w_hat)
+        assert not (ratio <= 1.0 and fro <= 2e-3), (shared, ratio, fro)
 
 
 @pytest.mark.parametrize("shape", list(synthetic.DECODE_SHAPES))
