@@ -36,6 +36,13 @@ METRIC = "W4A4 NVFP4 GEMM TFLOPS incl. act-quant (M=8192)"
 UNIT = "TFLOPS"
 
 
+# Dense FP4 rate measured on this machine's B200s by --probe-peaks (block-scaled
+# M128 N256 K64 MMAs back to back from shared memory on all 148 SMs, 5 ms,
+# clocks under the power cap): a second roofline denominator beside 4 x the
+# measured BF16 burst.
+PROBE_FP4_TFLOPS = 8141.0
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -43,6 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--m", type=int, default=8192)
+    ap.add_argument("--gemm-kernel", choices=["auto", "pair"], default="auto",
+                    help="large-M kernel of the headline step: AUTO's choice, or the CTA-pair kernel")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode GB/s sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mlp", action="store_true", help="skip the prefill and long-prefill MLP measurements")
@@ -268,21 +277,22 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     flops = 2.0 * p.m * p.n * p.k
     stream = torch.cuda.current_stream(device)
+    gemm_flags = nv.NVFP4_GEMM_FORCE_LARGE_PAIR if args.gemm_kernel == "pair" else nv.NVFP4_GEMM_AUTO
 
     def step(ev):
+        # nothing between the two launches: the GEMM (programmatic dependent
+        # launch) starts its weight loads under the quantiser's tail
         if ev is not None:
             ev[0].record(stream)
         nv.quantize_act(a_dev, act_scale=act_scale, out=aq)
+        nv.gemm(aq, fw, out=c, flags=gemm_flags)
         if ev is not None:
             ev[1].record(stream)
-        nv.gemm(aq, fw, out=c)
-        if ev is not None:
-            ev[2].record(stream)
 
     for _ in range(args.warmup):
         step(None)
         flush.zero_()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     torch.cuda.synchronize(device)
     if world > 1:
         dist.barrier()
@@ -298,9 +308,23 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(device)
-    step_ms = [e[0].elapsed_time(e[2]) for e in events]
-    gemm_ms = [e[1].elapsed_time(e[2]) for e in events]
-    quant_ms = [e[0].elapsed_time(e[1]) for e in events]
+    step_ms = [e[0].elapsed_time(e[1]) for e in events]
+    # the two kernels of the step, each timed alone (events around it, L2
+    # flushed before each), for the roofline of the GEMM and the quantiser's GB/s
+    split = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda._sleep(2_000_000)
+    for i in range(args.steps):
+        split[i][0].record(stream)
+        nv.quantize_act(a_dev, act_scale=act_scale, out=aq)
+        split[i][1].record(stream)
+        flush.zero_()
+        split[i][2].record(stream)
+        nv.gemm(aq, fw, out=c, flags=gemm_flags)
+        split[i][3].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(device)
+    quant_ms = [e[0].elapsed_time(e[1]) for e in split]
+    gemm_ms = [e[2].elapsed_time(e[3]) for e in split]
     total_ms, value = aggregate_over_ranks(sum(step_ms), flops, args.steps, world, device)
     ms_per_step = total_ms / args.steps
     qs = sorted(step_ms)
@@ -312,14 +336,20 @@ def run_ours(args):
     achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak, "traffic": profiled_traffic(),
-                "kernel": "gemm_large_kernel",
+                "kernel": "gemm_pair_kernel" if args.gemm_kernel == "pair" else "gemm_large_kernel",
                 "peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/BF16 nominal)",
-                "datasheet_fp4_frac": achieved / 9000.0}
+                "datasheet_fp4_frac": achieved / 9000.0,
+                "probe_fp4_frac": achieved / PROBE_FP4_TFLOPS,
+                "probe_fp4_basis": f"{PROBE_FP4_TFLOPS} TFLOP/s: back-to-back M128 N256 K64 block-scaled FP4 MMAs from "
+                                   "shared memory on every SM over 5 ms (--probe-peaks on this pool's B200s)",
+                "timing": "GEMM launched alone between events, L2 flushed before it"}
     quant_avg_ms = statistics.mean(quant_ms)
     quant_bytes = p.m * p.k * 2 + p.m * p.k // 2 + p.m * p.k // 16
     extra = {"act_quant": {"ms": quant_avg_ms, "GB/s": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
-                           "frac_hbm": quant_bytes / (quant_avg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-             "gemm_ms": gemm_avg_ms}
+                           "frac_hbm": quant_bytes / (quant_avg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                           "timing": "launched alone between events, L2 flushed before it"},
+             "gemm_ms": gemm_avg_ms,
+             "step_minus_gemm_us": (statistics.median(step_ms) - statistics.median(gemm_ms)) * 1e3}
 
     result = {}
     if not args.profile_gemm:

@@ -19,10 +19,10 @@
 //    warp-specialised, 128 x 256 tiles; gemm_pair_kernel, the same on CTA
 //    pairs (cta_group::2) with 256 x 256 tiles.
 //  * gemm_decode.cuh: gemm_decode_kernel, small M (<= 64 tokens), bound by
-//    streaming the weight.  Stream-K: the (256-column tile, 256-deep k-tile)
+//    streaming the weight.  Stream-K: the (128-column tile, 256-deep k-tile)
 //    units are split evenly over one CTA per SM; a tile whose k-range spans
-//    several CTAs is reduced by all of them, each summing a column slice of
-//    the FP32 partials in CTA order, so the result is deterministic.
+//    several CTAs is finished by the CTA holding its first k-tile, which adds
+//    the others' FP32 partials in CTA order, so the result is deterministic.
 #pragma once
 
 #include <cuda.h>
@@ -56,7 +56,7 @@ struct GemmParams {
     // decode kernel (stream-K): work units = w_tiles x k_tiles, split evenly
     // over `ctas` co-resident CTAs; partial tiles meet in `ws`
     int units, ctas;
-    uint8_t* ws;                // [MAX_CTAS][2][BT][256] tagged partial-tile words
+    uint8_t* ws;                // [MAX_CTAS][BT][128] tagged partial-tile words
     unsigned long long epoch;   // this call's value; its low 32 bits tag the partial words
     // decode kernel with the activation quantisation fused in: the raw
     // activations (act_scale == nullptr: dynamic scale amax/2688, computed by

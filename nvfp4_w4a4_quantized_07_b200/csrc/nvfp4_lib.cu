@@ -269,8 +269,11 @@ nvfp4_status launch_quant(const QuantParams& p, cudaStream_t s, QuantKind kind =
         l.row_begin = r0;
         l.total = (uint32_t)(rows * pairs);
         const unsigned blocks = (unsigned)((l.total + kQuantThreads - 1) / kQuantThreads);
-        if (kind == kQuantPlain)
-            quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, l);
+        if (kind == kQuantPlain && !p.in_fp32)
+            quantize_kernel<2, false><<<(unsigned)((l.total + kQuantThreads * 2 - 1) / (kQuantThreads * 2)),
+                                        kQuantThreads, 0, s>>>(p, l);
+        else if (kind == kQuantPlain)
+            quantize_kernel<1, true><<<blocks, kQuantThreads, 0, s>>>(p, l);
         else if (kind == kQuantSiluMul)
             silu_mul_quantize_kernel<<<blocks, kQuantThreads, 0, s>>>(p, *sp, l);
         else

@@ -237,49 +237,75 @@ __device__ __forceinline__ void quantize_pair_store(const QuantParams& p, const 
     }
 }
 
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p,
-                                                               const QuantLaunch l)
+// Each thread quantises ITEMS (row, block pair) items, 256 threads apart,
+// and issues the loads of all of them before any arithmetic: two BF16 items
+// keep 128 bytes of input in flight per thread within the register budget of
+// four resident blocks (a streaming kernel is bound by the bytes in flight
+// per SM).  FP32 input (64 bytes per item) takes one item per thread.
+constexpr int kQuantMinBlocks = 4;
+
+template <int ITEMS, bool FP32>
+__global__ void __launch_bounds__(kQuantThreads, kQuantMinBlocks) quantize_kernel(const __grid_constant__ QuantParams p,
+                                                                                const QuantLaunch l)
 {
-    const uint32_t t = blockIdx.x * kQuantThreads + threadIdx.x;
-    const bool mapped = t < l.total;
-    const uint32_t rl = mapped ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
-    const uint32_t pr = mapped ? t - rl * l.pairs : 0u;
-    const int64_t r = l.row_begin + rl;
+    constexpr int kQuantItems = ITEMS;
+    // A GEMM launched after this kernel with programmatic dependent launch may
+    // start now (it loads weights until this kernel has completed).
+    if (threadIdx.x == 0) launch_dependents();
+    const uint32_t t_first = blockIdx.x * (kQuantThreads * kQuantItems) + threadIdx.x;
     const int64_t nb = p.k >> 4;
-    const int64_t kb0 = (int64_t)pr * 2;
-    const bool row_live = mapped && r < p.rows;
-    const bool live0 = row_live && kb0 < nb;
-    const bool live1 = row_live && kb0 + 1 < nb;
-
     const float s_g = load_scale(p);
-    if (p.scale_out != nullptr && t == 0 && l.row_begin == 0) *p.scale_out = s_g;
+    if (p.scale_out != nullptr && t_first == 0 && l.row_begin == 0) *p.scale_out = s_g;
 
-    // Issue every load of both blocks before any arithmetic.
-    float v0[16], v1[16];
-    if (p.in_fp32) {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + r * p.ldx + kb0 * 16);
-        float4 f[8];
+    bool mapped[kQuantItems], live0[kQuantItems], live1[kQuantItems];
+    uint32_t pr[kQuantItems];
+    int64_t r[kQuantItems], kb0[kQuantItems];
+    uint4 u[kQuantItems][FP32 ? 8 : 4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            f[j] = ((j < 4) ? live0 : live1) ? __ldcs(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < kQuantItems; ++i) {
+        const uint32_t t = t_first + i * kQuantThreads;
+        mapped[i] = t < l.total;
+        const uint32_t rl = mapped[i] ? __umulhi(t << 2, l.div_mul) >> l.div_shift : 0u;
+        pr[i] = mapped[i] ? t - rl * l.pairs : 0u;
+        r[i] = l.row_begin + rl;
+        kb0[i] = (int64_t)pr[i] * 2;
+        const bool row_live = mapped[i] && r[i] < p.rows;
+        live0[i] = row_live && kb0[i] < nb;
+        live1[i] = row_live && kb0[i] + 1 < nb;
+        if (FP32) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) + r[i] * p.ldx + kb0[i] * 16);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v0[4 * j] = f[j].x; v0[4 * j + 1] = f[j].y; v0[4 * j + 2] = f[j].z; v0[4 * j + 3] = f[j].w;
-            v1[4 * j] = f[4 + j].x; v1[4 * j + 1] = f[4 + j].y; v1[4 * j + 2] = f[4 + j].z; v1[4 * j + 3] = f[4 + j].w;
+            for (int j = 0; j < 8; ++j) u[i][j] = ((j < 4) ? live0[i] : live1[i]) ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+        } else {
+            const uint4* src =
+                reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r[i] * p.ldx + kb0[i] * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) u[i][j] = ((j < 2) ? live0[i] : live1[i]) ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
         }
-    } else {
-        const uint4* src =
-            reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.x) + r * p.ldx + kb0 * 16);
-        uint4 u[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) u[j] = ((j < 2) ? live0 : live1) ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
-        unpack_bf16x8(u[0], v0);
-        unpack_bf16x8(u[1], v0 + 8);
-        unpack_bf16x8(u[2], v1);
-        unpack_bf16x8(u[3], v1 + 8);
     }
-
-    quantize_pair_store(p, l, mapped, pr, r, kb0, live0, live1, s_g, v0, v1);
+#pragma unroll
+    for (int i = 0; i < kQuantItems; ++i) {
+        float v0[16], v1[16];
+        if (FP32) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v0[4 * j] = __uint_as_float(u[i][j].x);
+                v0[4 * j + 1] = __uint_as_float(u[i][j].y);
+                v0[4 * j + 2] = __uint_as_float(u[i][j].z);
+                v0[4 * j + 3] = __uint_as_float(u[i][j].w);
+                v1[4 * j] = __uint_as_float(u[i][4 + j].x);
+                v1[4 * j + 1] = __uint_as_float(u[i][4 + j].y);
+                v1[4 * j + 2] = __uint_as_float(u[i][4 + j].z);
+                v1[4 * j + 3] = __uint_as_float(u[i][4 + j].w);
+            }
+        } else {
+            unpack_bf16x8(u[i][0], v0);
+            unpack_bf16x8(u[i][1], v0 + 8);
+            unpack_bf16x8(u[i][2], v1);
+            unpack_bf16x8(u[i][3], v1 + 8);
+        }
+        quantize_pair_store(p, l, mapped[i], pr[i], r[i], kb0[i], live0[i], live1[i], s_g, v0, v1);
+    }
 }
 
 // ---------------------------------------------------------------------------
