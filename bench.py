@@ -65,6 +65,13 @@ def parse():
                     help="with --decode-case: time nvfp4_linear_decode (quantisation fused in)")
     ap.add_argument("--decode-case", default=None,
                     help="time one decode GEMM only, e.g. m16_5120x5120 (for ncu captures)")
+    ap.add_argument("--kv-case", action="store_true",
+                    help="time the FP8 KV-cache kernel alone on 8192 tokens x 1024 (for ncu captures)")
+    ap.add_argument("--swiglu-case", choices=["fused", "plain"], default=None,
+                    help="time the 8192-token gate/up GEMM (34816 x 5120) with the SwiGLU-quantise epilogue "
+                         "(fused) or with the BF16 output (plain), for ncu captures")
+    ap.add_argument("--prefill-case", action="store_true",
+                    help="time the 4096 x 5120 x 5120 prefill projection: quantiser, GEMM and both (--gemm-kernel)")
     ap.add_argument("--short-kernels", action="store_true",
                     help="per-launch times of the short kernels (decode GEMMs at m=16, the FP8 KV cache at 8192 "
                          "tokens) from back-to-back launches over rotating inputs larger than L2")
@@ -697,6 +704,111 @@ def run_glue_case(args):
     return 0
 
 
+def _case_ms(fn, args, flush, stream, device):
+    """Median CUDA-event time (ms) of ``fn`` over ``args.steps`` launches after
+    ``args.warmup``, L2 flushed before each."""
+    import torch
+    times = []
+    for it in range(args.warmup + args.steps):
+        flush.zero_()
+        torch.cuda._sleep(400_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def _case_setup():
+    import torch
+
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    from nvfp4_w4a4_quantized_07_b200 import build as nvbuild
+    nvbuild.build()
+    nv.load()
+    device = torch.device("cuda", 0)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    return nv, device, flush, torch.cuda.current_stream(device)
+
+
+def run_kv_case(args):
+    """One layer's new K and V rows (8192 tokens x 1024, BF16) quantised to FP8
+    and scattered into shuffled slots of a 16384-slot cache, L2 flushed before
+    each launch."""
+    import torch
+
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+    nv, device, flush, stream = _case_setup()
+    tokens = 8192
+    k_rows, v_rows = (t.to(device) for t in synthetic.kv_rows(tokens, seed=11))
+    ks = torch.empty(1, dtype=torch.float32, device=device)
+    vs = torch.empty(1, dtype=torch.float32, device=device)
+    nv.fp8_calibrate(k_rows, torch.zeros(1, dtype=torch.float32, device=device), ks)
+    nv.fp8_calibrate(v_rows, torch.zeros(1, dtype=torch.float32, device=device), vs)
+    slots = torch.randperm(2 * tokens, generator=torch.Generator().manual_seed(0))[:tokens].to(device)
+    kc = torch.empty((2 * tokens, k_rows.shape[1]), dtype=torch.uint8, device=device)
+    vc = torch.empty_like(kc)
+    ms = _case_ms(lambda: nv.kv_cache_quantize_fp8(k_rows, v_rows, ks, vs, kc, vc, slots), args, flush, stream,
+                  device)
+    nbytes = 2 * k_rows.numel() * 3 + tokens * 8
+    print(json.dumps({"kv_case": f"{tokens}x{k_rows.shape[1]}", "us": ms * 1e3,
+                      "GB/s": nbytes / (ms * 1e-3) / 1e9, "steps": args.steps}), flush=True)
+    return 0
+
+
+def run_swiglu_case(args):
+    """The MLP gate/up GEMM on 8192 tokens (fused [gate; up] weight 34816 x
+    5120, two modules): with the SwiGLU-quantise epilogue or the plain BF16
+    output, L2 flushed before each launch."""
+    import torch
+
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+    nv, device, flush, stream = _case_setup()
+    p = synthetic.mlp_gate_up(m=8192)
+    fw = nv.quantize_weight([w.to(device) for w in p.modules])
+    aq = nv.quantize_act(p.a.to(device))
+    f = synthetic.MLP_INTERMEDIATE
+    if args.swiglu_case == "fused":
+        h_scale = torch.tensor([0.01], dtype=torch.float32, device=device)
+        hq = nv.gemm_swiglu_quantize(aq, fw, h_scale)
+        fn = lambda: nv.gemm_swiglu_quantize(aq, fw, h_scale, out=hq)  # noqa: E731
+    else:
+        c = torch.empty((p.m, 2 * f), dtype=torch.bfloat16, device=device)
+        fn = lambda: nv.gemm(aq, fw, out=c)  # noqa: E731
+    ms = _case_ms(fn, args, flush, stream, device)
+    print(json.dumps({"swiglu_case": args.swiglu_case, "m": p.m, "n": 2 * f, "k": p.k, "ms": ms,
+                      "TFLOPS": 2.0 * p.m * 2 * f * p.k / (ms * 1e-3) / 1e12, "steps": args.steps}), flush=True)
+    return 0
+
+
+def run_prefill_case(args):
+    """The 4096 x 5120 x 5120 prefill projection: the quantiser alone, the GEMM
+    alone and the two together, L2 flushed before each."""
+    import torch
+
+    from nvfp4_w4a4_quantized_07_b200 import synthetic
+    nv, device, flush, stream = _case_setup()
+    p = synthetic.prefill()
+    a = p.a.to(device)
+    fw = nv.quantize_weight([w.to(device) for w in p.modules])
+    s_a = nv.quantize_act(a).scale.clone()
+    aq = nv.quantize_act(a, act_scale=s_a)
+    c = torch.empty((p.m, p.n), dtype=torch.bfloat16, device=device)
+    flags = nv.NVFP4_GEMM_FORCE_LARGE_PAIR if args.gemm_kernel == "pair" else nv.NVFP4_GEMM_AUTO
+    quant = lambda: nv.quantize_act(a, act_scale=s_a, out=aq)  # noqa: E731
+    gemm = lambda: nv.gemm(aq, fw, out=c, flags=flags)  # noqa: E731
+    res = {"prefill_case": f"{p.m}x{p.k}x{p.n}", "gemm_kernel": args.gemm_kernel,
+           "quant_ms": _case_ms(quant, args, flush, stream, device),
+           "gemm_ms": _case_ms(gemm, args, flush, stream, device),
+           "step_ms": _case_ms(lambda: (quant(), gemm()), args, flush, stream, device), "steps": args.steps}
+    res["TFLOPS"] = 2.0 * p.m * p.n * p.k / (res["step_ms"] * 1e-3) / 1e12
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def run_decode_case(args):
     """One decode-shaped GEMM (``m<M>_<shape>``), L2 flushed before each launch."""
     import torch
@@ -880,6 +992,12 @@ def main():
         return run_decode_case(args)
     if args.short_kernels:
         return run_short_kernels(args)
+    if args.kv_case:
+        return run_kv_case(args)
+    if args.swiglu_case:
+        return run_swiglu_case(args)
+    if args.prefill_case:
+        return run_prefill_case(args)
     if args.probe_peaks:
         return run_probe_peaks(args)
     if args.glue_case:
