@@ -50,8 +50,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--m", type=int, default=8192)
-    ap.add_argument("--gemm-kernel", choices=["auto", "pair"], default="auto",
-                    help="large-M kernel of the headline step: AUTO's choice, or the CTA-pair kernel")
+    ap.add_argument("--gemm-kernel", choices=["auto", "single", "pair"], default="auto",
+                    help="large-M kernel: AUTO's choice, the single-CTA kernel or the CTA-pair kernel")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode GB/s sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-mlp", action="store_true", help="skip the prefill and long-prefill MLP measurements")
@@ -93,6 +93,11 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+GEMM_FLAGS = {"auto": lambda nv: nv.NVFP4_GEMM_AUTO, "single": lambda nv: nv.NVFP4_GEMM_FORCE_LARGE,
+              "pair": lambda nv: nv.NVFP4_GEMM_FORCE_LARGE_PAIR}
+KERNEL_NAMES = {1: "gemm_large_kernel", 2: "gemm_decode_kernel", 3: "gemm_pair_kernel"}
+
+
 def kernel_source_hash() -> str:
     """Hash of the large-M GEMM kernel's device source (the counters of a
     profile hold only for the source they were taken on)."""
@@ -103,11 +108,13 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per launch of the GEMM from the committed ncu summary
-    (``source_hash:`` and ``dram_bytes_per_launch:`` lines), if it was taken on
-    the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "gemm_large_gdn_in_proj_8192.md")
+def profiled_traffic(kernel: str = "gemm_large_kernel"):
+    """DRAM bytes per launch of the GEMM from the committed ncu summary of that
+    kernel (``source_hash:`` and ``dram_bytes_per_launch:`` lines), if it was
+    taken on the current kernel source; else None."""
+    name = {"gemm_large_kernel": "gemm_large_gdn_in_proj_8192.md",
+            "gemm_pair_kernel": "gemm_pair_gdn_in_proj_8192.md"}[kernel]
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     fields = {}
@@ -284,11 +291,12 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     flops = 2.0 * p.m * p.n * p.k
     stream = torch.cuda.current_stream(device)
-    gemm_flags = nv.NVFP4_GEMM_FORCE_LARGE_PAIR if args.gemm_kernel == "pair" else nv.NVFP4_GEMM_AUTO
+    gemm_flags = GEMM_FLAGS[args.gemm_kernel](nv)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    kernel_name = KERNEL_NAMES[nv.gemm_kernel_for(p.m, p.n, sms, gemm_flags)]
 
     def step(ev):
-        # nothing between the two launches: the GEMM (programmatic dependent
-        # launch) starts its weight loads under the quantiser's tail
+        # the quantiser and the GEMM back to back on one stream, nothing between
         if ev is not None:
             ev[0].record(stream)
         nv.quantize_act(a_dev, act_scale=act_scale, out=aq)
@@ -342,8 +350,8 @@ def run_ours(args):
     gemm_avg_ms = statistics.mean(gemm_ms)
     achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp4_peak, "traffic": profiled_traffic(),
-                "kernel": "gemm_pair_kernel" if args.gemm_kernel == "pair" else "gemm_large_kernel",
+                "frac": achieved / fp4_peak, "traffic": profiled_traffic(kernel_name),
+                "kernel": kernel_name,
                 "peak_basis": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (FP4/BF16 nominal)",
                 "datasheet_fp4_frac": achieved / 9000.0,
                 "probe_fp4_frac": achieved / PROBE_FP4_TFLOPS,
@@ -467,6 +475,13 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
     out["dynamic_act_scale"] = {"value": 2.0 * p.m * p.n * p.k / (dyn_ms * 1e-3) / 1e12, "unit": UNIT,
                                 "ms_per_step": dyn_ms}
 
+    # ---- the same layer as one launch (static scale quantised inside the
+    # large-M kernel), L2 flushed before each
+    fused_ms = _timed(lambda: nv.linear_prefill(a_dev, fw, act_scale, out=c, a_out=aq), flush, stream, device)
+    out["one_launch_layer"] = {"value": 2.0 * p.m * p.n * p.k / (fused_ms * 1e-3) / 1e12, "unit": UNIT,
+                               "ms_per_step": fused_ms,
+                               "call": "nvfp4_linear_prefill (bit-identical to the two launches)"}
+
     # ---- the same GEMM with the Gated DeltaNet gates computed in its epilogue
     # from the last two (head-wide) segments, against the plain GEMM
     if len(p.widths) >= 2 and p.widths[-1] == p.widths[-2]:
@@ -475,7 +490,8 @@ def extra_measurements(args, p, a_dev, fw, act_scale, c, flush, device, stream, 
         g = torch.empty((p.m, heads), dtype=torch.float32, device=device)
         beta = torch.empty_like(g)
         a_col = p.n - 2 * heads
-        ms_plain = _timed(lambda: nv.gemm(aq, fw, out=c), flush, stream, device)
+        # against the same (single-CTA) kernel without the gates
+        ms_plain = _timed(lambda: nv.gemm(aq, fw, out=c, flags=nv.NVFP4_GEMM_FORCE_LARGE), flush, stream, device)
         ms_gdn = _timed(lambda: nv.gemm_gdn(aq, fw, a_col, a_col + heads, A_log, dt_bias, out=c, g=g, beta=beta),
                         flush, stream, device)
         out["gdn_gate_epilogue"] = {"heads": heads, "gemm_ms": ms_plain, "gemm_gdn_ms": ms_gdn,
@@ -540,6 +556,11 @@ def prefill_and_mlp_measurements(flush, device, stream, nv, synthetic, peaks):
     ms = _timed(prefill_step, flush, stream, device)
     flops = 2.0 * p.m * p.n * p.k
     res["prefill_4096x5120x5120"] = {"value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms}
+    # the same layer as one launch (quantisation fused into the large-M kernel)
+    fused_ms = _timed(lambda: nv.linear_prefill(a, fw, s_a, out=c, a_out=aq), flush, stream, device)
+    res["prefill_4096x5120x5120"]["one_launch"] = {
+        "value": flops / (fused_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": fused_ms,
+        "call": "nvfp4_linear_prefill (static scale; bit-identical to the two launches)"}
     del a, fw, aq, c
 
     # ---- long-prefill MLP
@@ -797,7 +818,7 @@ def run_prefill_case(args):
     s_a = nv.quantize_act(a).scale.clone()
     aq = nv.quantize_act(a, act_scale=s_a)
     c = torch.empty((p.m, p.n), dtype=torch.bfloat16, device=device)
-    flags = nv.NVFP4_GEMM_FORCE_LARGE_PAIR if args.gemm_kernel == "pair" else nv.NVFP4_GEMM_AUTO
+    flags = GEMM_FLAGS[args.gemm_kernel](nv)
     quant = lambda: nv.quantize_act(a, act_scale=s_a, out=aq)  # noqa: E731
     gemm = lambda: nv.gemm(aq, fw, out=c, flags=flags)  # noqa: E731
     res = {"prefill_case": f"{p.m}x{p.k}x{p.n}", "gemm_kernel": args.gemm_kernel,

@@ -77,7 +77,9 @@ typedef struct {
 #define NVFP4_MAX_SEGMENTS 16
 
 /* nvfp4_gemm flags */
-#define NVFP4_GEMM_AUTO 0u              /* decode kernel for m <= 64, large kernel otherwise */
+#define NVFP4_GEMM_AUTO 0u              /* decode kernel for m <= 64; otherwise the CTA-pair kernel when
+                                           it needs no more waves of tiles than the single-CTA kernel
+                                           (m >= 256, no gate outputs), else the single-CTA kernel */
 #define NVFP4_GEMM_FORCE_LARGE 1u       /* the persistent large-M kernel (one CTA per SM, 128 x 256 tiles) */
 #define NVFP4_GEMM_FORCE_DECODE 2u      /* the split-K decode kernel (m <= 64) */
 #define NVFP4_GEMM_FORCE_LARGE_PAIR 3u  /* the large-M kernel on CTA pairs (cta_group::2, 256 x 256 tiles) */
@@ -110,6 +112,13 @@ NVFP4_API size_t nvfp4_quant_workspace_size(void);
  * (consecutive calls on one stream may share it: a decode kernel touches the
  * workspace only after the previous kernel in the stream has completed). */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags);
+
+/* The kernel nvfp4_gemm runs for an m x n output with these flags on a device
+ * with `sms` streaming multiprocessors: NVFP4_GEMM_FORCE_DECODE,
+ * NVFP4_GEMM_FORCE_LARGE or NVFP4_GEMM_FORCE_LARGE_PAIR (the flag that selects
+ * it), or -1 for out-of-range arguments.  with_gates: the nvfp4_gemm_gdn form.
+ * A pure host function (no CUDA calls). */
+NVFP4_API int nvfp4_gemm_kernel_for(int64_t m, int64_t n, int sms, uint32_t flags, int with_gates);
 
 /* ------------------------------------------------------------------------
  * nvfp4_quantize_weight - offline, per module (post-training, calibration
@@ -296,6 +305,53 @@ NVFP4_API nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int
                                  const float* act_scale_dev, float* act_scale_out_dev, const uint8_t* w_q,
                                  const uint8_t* w_sf, int64_t n, const nvfp4_segment* segs, int nsegs, void* c,
                                  nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * nvfp4_linear_prefill - one W4A4 linear layer for m > 64 tokens in a single
+ * launch: the activations are quantised to NVFP4 with the static
+ * (calibrated) scale inside the large-M GEMM kernel and multiplied with the
+ * fused NVFP4 weight, with the per-segment scale epilogue ("Why Gated
+ * DeltaNet Survives 4-Bit Quantization": W4A4 with on-the-fly activation
+ * quantisation, abstract; per-module global scales, abstract, last
+ * sentence).  The first m-blocks of A are quantised before the first MMAs,
+ * the rest while the MMAs run (tiles are scheduled in bands of 8 m-blocks).
+ * a_q / a_sf receive exactly the bytes nvfp4_quantize_act writes with the
+ * same scale, and c exactly what nvfp4_gemm (NVFP4_GEMM_FORCE_LARGE) writes
+ * from them.
+ *
+ *   a, dt, m, k, lda  raw activations as for nvfp4_quantize_act; BF16 only
+ *                     (UNSUPPORTED otherwise); m > 64 (m <= 64: UNSUPPORTED,
+ *                     use nvfp4_linear_decode; m == 0 is a no-op).
+ *   act_scale_dev     device FP32 decode scale of A (required: static mode).
+ *   a_q, a_sf         device outputs as for nvfp4_quantize_act (the kernel's
+ *                     own staging of the quantised A; the caller may reuse it).
+ *   w_q, w_sf, n, segs, nsegs, c, odt, ldc   as for nvfp4_gemm.
+ *   workspace         device, >= nvfp4_linear_prefill_workspace_size(m)
+ *                     bytes, 16-byte aligned: one 8-byte ready word per 128
+ *                     rows of A, tagged per call with a tag that grows from
+ *                     call to call in this process.  ZERO IT ONCE before its
+ *                     first use (after that, consecutive calls on one stream
+ *                     may share it without clearing; calls that may run
+ *                     concurrently must not).
+ * The kernel is persistent (one CTA per SM) and its CTAs wait (bounded) on
+ * one another's quantised rows, so it needs the whole GPU to itself to make
+ * progress at full speed; a wait that runs out sets the device status
+ * (nvfp4_check_device_status returns NVFP4_ERR_TIMEOUT).
+ *
+ * Performance: on B200 this single launch is currently SLOWER than
+ * nvfp4_quantize_act followed by nvfp4_gemm: 0.272 ms against 0.259-0.265 ms
+ * for 8192 x 5120 x 12384, 0.084 ms against 0.077-0.079 ms for
+ * 4096 x 5120 x 5120.  Quantising the first 8-16 m-blocks before the first
+ * MMA costs 6-10 us, the two background warps quantise about 0.5 TB/s (a
+ * band of 8 m-blocks per ~20 us, late for the 4096-row case), and the banded
+ * tile order and the background traffic slow the mainloop by ~4 %.  Use it
+ * where one launch per layer matters more than the last few percent.
+ * ---------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_linear_prefill_workspace_size(int64_t m);
+NVFP4_API nvfp4_status nvfp4_linear_prefill(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                  const float* act_scale_dev, uint8_t* a_q, uint8_t* a_sf, const uint8_t* w_q,
+                                  const uint8_t* w_sf, int64_t n, const nvfp4_segment* segs, int nsegs, void* c,
+                                  nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * nvfp4_silu_mul_quantize - the glue of a gated (SwiGLU) MLP whose gate/up

@@ -27,8 +27,10 @@ NVFP4_MAX_SEGMENTS = 16
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CUDA", 5: "TIMEOUT",
                 6: "WORKSPACE"}
 EXPORTED = ("nvfp4_sf_bytes", "nvfp4_sf_offset", "nvfp4_quant_workspace_size", "nvfp4_gemm_workspace_size",
+            "nvfp4_gemm_kernel_for",
             "nvfp4_quantize_weight", "nvfp4_quantize_act", "nvfp4_silu_mul_quantize", "nvfp4_gemm",
-            "nvfp4_linear_decode", "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc", "nvfp4_gemm_gdn",
+            "nvfp4_linear_decode", "nvfp4_linear_prefill", "nvfp4_linear_prefill_workspace_size",
+            "nvfp4_gemm_swiglu_quantize", "nvfp4_gemm_decode_noalloc", "nvfp4_gemm_gdn",
             "nvfp4_fp8_calibrate", "nvfp4_kv_cache_quantize_fp8",
             "nvfp4_get_last_error_string", "nvfp4_check_device_status", "nvfp4_selftest_wait_timeout",
             "nvfp4_version")
@@ -71,6 +73,8 @@ def load():
     L.nvfp4_quant_workspace_size.restype = SZ
     L.nvfp4_gemm_workspace_size.argtypes = [I64, I64, I64, U32]
     L.nvfp4_gemm_workspace_size.restype = SZ
+    L.nvfp4_gemm_kernel_for.argtypes = [I64, I64, INT, U32, INT]
+    L.nvfp4_gemm_kernel_for.restype = INT
     L.nvfp4_quantize_weight.argtypes = [P, INT, I64, I64, I64, I64, I64, P, P, P, P, P, SZ, P]
     L.nvfp4_quantize_weight.restype = INT
     L.nvfp4_quantize_act.argtypes = [P, INT, I64, I64, I64, P, P, P, P, P, SZ, P]
@@ -91,6 +95,11 @@ def load():
     L.nvfp4_linear_decode.argtypes = [P, INT, I64, I64, I64, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P, INT,
                                       I64, P, SZ, P]
     L.nvfp4_linear_decode.restype = INT
+    L.nvfp4_linear_prefill.argtypes = [P, INT, I64, I64, I64, P, P, P, P, P, I64, ctypes.POINTER(Segment), INT, P,
+                                       INT, I64, P, SZ, P]
+    L.nvfp4_linear_prefill.restype = INT
+    L.nvfp4_linear_prefill_workspace_size.argtypes = [I64]
+    L.nvfp4_linear_prefill_workspace_size.restype = SZ
     L.nvfp4_gemm_decode_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, ctypes.POINTER(Segment), INT, P, INT, I64,
                                             P]
     L.nvfp4_gemm_decode_noalloc.restype = INT
@@ -467,6 +476,49 @@ def linear_decode(a, w: FusedWeight, act_scale=None, out_dtype=None, out=None, w
     return out
 
 
+_prefill_ws_cache: dict = {}
+
+
+def linear_prefill(a, w: FusedWeight, act_scale, out_dtype=None, out=None, a_out: QuantizedActivation | None = None,
+                   workspace=None):
+    """``nvfp4_linear_prefill``: one W4A4 layer for m > 64 tokens in one
+    launch (the static-scale activation quantisation fused into the large-M
+    GEMM).  ``act_scale``: 1-element FP32 device scale.  ``a_out`` receives the
+    quantised activations (allocated when not given).  Returns
+    ``(out, a_out)``."""
+    import torch
+    _require_cuda(a, act_scale)
+    if a.dim() != 2 or a.stride(1) != 1:
+        raise ValueError("activations must be a 2-D tensor with unit column stride")
+    m, k = a.shape
+    if k != w.k:
+        raise ValueError("K mismatch between activations and weight")
+    L = load()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out is None:
+        out = torch.empty((m, w.n), dtype=out_dtype, device=a.device)
+    odt = {torch.bfloat16: NVFP4_OUT_BF16, torch.float32: NVFP4_OUT_FP32}[out.dtype]
+    if a_out is None:
+        a_out = QuantizedActivation(
+            q=torch.empty((m, k // 2), dtype=torch.uint8, device=a.device),
+            sf=torch.empty(max(L.nvfp4_sf_bytes(m, k), 1), dtype=torch.uint8, device=a.device),
+            scale=act_scale, m=m, k=k)
+    if workspace is None:
+        need = max(int(L.nvfp4_linear_prefill_workspace_size(m)), 16)
+        key = (a.device.index if a.device.index is not None else torch.cuda.current_device())
+        ws = _prefill_ws_cache.get(key)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(need, dtype=torch.uint8, device=a.device)   # zeroed once, as the call requires
+            _prefill_ws_cache[key] = ws
+        workspace = ws
+    arr = segment_array(w.segments)
+    _check("nvfp4_linear_prefill", L.nvfp4_linear_prefill(
+        _ptr(a), _in_dtype(a), m, k, a.stride(0), _ptr(act_scale), _ptr(a_out.q), _ptr(a_out.sf), _ptr(w.q),
+        _ptr(w.sf), w.n, arr, len(w.segments), _ptr(out), odt, out.stride(0), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(out.device)))
+    return out, a_out
+
+
 def linear(a, w: FusedWeight, act_scale=None, out_dtype=None, flags: int = NVFP4_GEMM_AUTO):
     """One W4A4 linear layer: quantise ``a`` on the fly, then the fused GEMM."""
     return gemm(quantize_act(a, act_scale), w, out_dtype=out_dtype, flags=flags)
@@ -478,3 +530,9 @@ def check_device_status(device=None):
 
 def version() -> int:
     return int(load().nvfp4_version())
+
+
+def gemm_kernel_for(m: int, n: int, sms: int, flags: int = NVFP4_GEMM_AUTO, with_gates: bool = False) -> int:
+    """``nvfp4_gemm_kernel_for``: the NVFP4_GEMM_FORCE_* value of the kernel
+    nvfp4_gemm runs for an m x n output on a device with ``sms`` SMs."""
+    return int(load().nvfp4_gemm_kernel_for(m, n, sms, flags, int(bool(with_gates))))

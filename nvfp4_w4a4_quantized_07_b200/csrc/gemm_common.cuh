@@ -84,6 +84,17 @@ struct GemmParams {
     // large-M kernel: tile i of the persistent schedule is tile (i + tile_shift)
     // mod the tile count (0 keeps the column-major order)
     int tile_shift;
+    // large-M kernel with the activation quantisation fused in: the raw BF16
+    // activations (a_in, lda) are quantised with the static scale *act_scale
+    // into qa_q / qa_sf (the buffers the A tensor map and a_sf point to);
+    // m-block j may be loaded once qa_ready[j] == (call tag << 32 | CTAs).
+    // The first qa_first m-blocks are quantised by every warp but the
+    // producer and the MMA issuer before the mainloop, the rest by warps 2-3
+    // while it runs.
+    uint8_t* qa_q;
+    uint8_t* qa_sf;
+    unsigned long long* qa_ready;
+    int qa_first;
 };
 
 __device__ __forceinline__ float segment_scale(const SegTable& t, int col)

@@ -175,6 +175,137 @@ static_assert(ACC1_COL + BN <= SF_COL && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COL
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace large
 
+// ---------------------------------------------------------------------------
+// Activation quantisation fused into the large-M kernel (QA): one launch
+// quantises the raw BF16 activations and multiplies them.  The tiles run in
+// bands of qa::BAND m-blocks (column-major inside a band), so the first wave
+// of tiles needs only the first m-blocks of A.  Those are quantised before the
+// mainloop by every warp but the producer and the MMA issuer, across all
+// CTAs; warps 2 and 3 then quantise the remaining m-blocks, in order, while
+// the MMAs run.  Each CTA counts itself into m-block j's ready word once its
+// share of j is stored; a producer loads rows of A only from m-blocks whose
+// word shows every CTA (the word carries a per-call tag that grows from call
+// to call; the workspace is zeroed once before its first use).  The
+// quantisation is quantize_kernel's, item for item, so
+// codes, scales and the GEMM output are bit-identical to the two launches.
+// ---------------------------------------------------------------------------
+namespace qa {
+constexpr int BAND = 8;            // m-blocks per band of the tile order
+constexpr int FIRST_ITEMS = 2;     // warp-chunks of 32 items in flight per lane, warps 2..15
+constexpr int BG_ITEMS = 4;        // the same, warps 2..3 (more bytes in flight for fewer warps)
+constexpr int FIRST_WARPS = 14;    // warps 2..15 quantise the first m-blocks
+constexpr int BG_WARPS = 2;        // warps 2..3 quantise the rest, a band at a time
+constexpr int BAR_FIRST = 8, BAR_BG = 9;  // named barriers
+}  // namespace qa
+
+// Tile t of the persistent schedule -> (m-block, n-block).
+template <bool QA>
+__device__ __forceinline__ void tile_mn(int t, const GemmParams& p, int& mb, int& nb)
+{
+    if (!QA) {
+        mb = t % p.m_tiles;
+        nb = t / p.m_tiles;
+        return;
+    }
+    const int band_tiles = qa::BAND * p.n_tiles;
+    const int band = t / band_tiles;
+    const int r = t - band * band_tiles;
+    const int bsz = min(qa::BAND, p.m_tiles - band * qa::BAND);
+    nb = r / bsz;
+    mb = band * qa::BAND + (r - nb * bsz);
+}
+
+// Quantise this warp's chunks of m-blocks [mb0, mb1): chunk c covers the 32
+// items (row, block pair) 32c' .. 32c' + 31 of m-block mb0 + c / (4 pairs),
+// c' = c mod (4 pairs), numbered row-major over its 128 rows x pairs (2 *
+// katoms) as in quantize_kernel, one item per lane.  The warp takes chunks c0,
+// c0 + stride, ..., ITEMS of them at a time with all their loads issued first.
+// Every lane fences its stores for the async proxy.
+template <int ITEMS>
+__device__ __forceinline__ void qa_quantize_range(const GemmParams& p, const QuantParams& qp, const QuantLaunch& ql,
+                                                  int mb0, int mb1, int c0, int stride, int lane, float s_g)
+{
+    const uint32_t pairs = ql.pairs;
+    const int per_mb = (int)(4u * pairs);    // 128 rows x pairs items / 32
+    const int chunks = (mb1 - mb0) * per_mb;
+    const int64_t nb16 = p.k >> 4;
+    for (int c = c0; c < chunks; c += stride * ITEMS) {
+        uint4 u[ITEMS][4];
+        bool have[ITEMS], live0[ITEMS], live1[ITEMS];
+        uint32_t pr[ITEMS];
+        int64_t r[ITEMS], kb0[ITEMS];
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int ci = c + i * stride;
+            have[i] = ci < chunks;               // the same for every lane
+            const int cc = have[i] ? ci : 0;
+            const int mbi = cc / per_mb;
+            const uint32_t item = (uint32_t)(cc - mbi * per_mb) * 32u + (uint32_t)lane;
+            const uint32_t rl = item / pairs;
+            pr[i] = item - rl * pairs;
+            r[i] = (int64_t)(mb0 + mbi) * 128 + rl;
+            kb0[i] = (int64_t)pr[i] * 2;
+            const bool row_live = have[i] && r[i] < p.m;
+            live0[i] = row_live && kb0[i] < nb16;
+            live1[i] = row_live && kb0[i] + 1 < nb16;
+            const uint4* src =
+                reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.a_in) + r[i] * p.lda + kb0[i] * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                u[i][j] = ((j < 2) ? live0[i] : live1[i]) ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            if (!have[i]) continue;
+            float v0[16], v1[16];
+            unpack_bf16x8(u[i][0], v0);
+            unpack_bf16x8(u[i][1], v0 + 8);
+            unpack_bf16x8(u[i][2], v1);
+            unpack_bf16x8(u[i][3], v1 + 8);
+            quantize_pair_store(qp, ql, true, pr[i], r[i], kb0[i], live0[i], live1[i], s_g, v0, v1);
+        }
+    }
+    fence_proxy_async_global();
+}
+
+// Count this CTA into m-block mb's ready word: the call tag in the high half
+// (raised to this call's by the maximum: tags grow from call to call and the
+// workspace starts at zero), CTAs done in the low half.  Two atomics, no
+// retry loop, so 148 CTAs marking one word cost 296 serialised updates.  The
+// caller has synchronised with every thread that stored part of this CTA's
+// share.
+__device__ __forceinline__ void qa_mark_ready(const GemmParams& p, int mb)
+{
+    unsigned long long* w = p.qa_ready + mb;
+    __threadfence();
+    atomicMax(w, (unsigned long long)(uint32_t)p.epoch << 32);
+    atomicAdd(w, 1ull);
+}
+
+// Warp-collective: wait (bounded) until m-blocks [ready_below, mb] are ready,
+// advancing ready_below over every ready m-block found (32 per look).  Then
+// the TMA loads this warp issues see the quantised rows.
+__device__ __forceinline__ bool qa_wait_ready(const GemmParams& p, int& ready_below, int mb, int lane)
+{
+    const unsigned long long want = ((unsigned long long)(uint32_t)p.epoch << 32) | gridDim.x;
+    const long long t0 = clock64();
+    while (ready_below <= mb) {
+        const int j = ready_below + lane;
+        const bool ok = j >= p.m_tiles || ld_volatile_u64(p.qa_ready + j) == want;
+        const unsigned bad = __ballot_sync(0xffffffffu, !ok);
+        ready_below = min(ready_below + (bad ? __ffs(bad) - 1 : 32), p.m_tiles);
+        if (ready_below > mb) break;
+        if (clock64() - t0 > kWaitCycles) {
+            if (lane == 0) record_status(kStatusTimeoutQuant);
+            return false;
+        }
+        __nanosleep(256);   // back off: 148 producers poll the same few words
+    }
+    __threadfence();
+    fence_proxy_async_global();
+    return true;
+}
+
 // SWIGLU: the gate/up GEMM of a gated MLP with its glue fused into the
 // epilogue.  Each 128 x 256 tile holds 128 gate columns (accumulator columns
 // 0..127) and the matching 128 up columns (128..255), loaded as two 128-row
@@ -182,7 +313,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // h = bf16(silu(bf16(g)) * bf16(u)) exactly as the unfused GEMM (BF16 output)
 // followed by silu_mul_quantize_kernel would, and quantises it with the
 // static scale h_scale, writing codes and tiled scales instead of C.
-template <bool SWIGLU>
+template <bool SWIGLU, bool QA = false>
 __global__ void __launch_bounds__(large::THREADS, 1)
     gemm_large_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ GemmParams p)
@@ -232,15 +363,47 @@ __global__ void __launch_bounds__(large::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_ptr;
 
+    if (QA && warp >= 2) {
+        // ------------------------------------------------------------ fused quantisation
+        const float s_g = *p.act_scale;
+        QuantParams qp = {};
+        qp.q = p.qa_q;
+        qp.sf = p.qa_sf;
+        qp.k = p.k;
+        QuantLaunch ql = {};
+        ql.pairs = 2u * (uint32_t)p.katoms;
+        // the first m-blocks, before the mainloop, by warps 2..15 of every CTA
+        qa_quantize_range<qa::FIRST_ITEMS>(p, qp, ql, 0, p.qa_first, blockIdx.x * qa::FIRST_WARPS + (warp - 2),
+                                           gridDim.x * qa::FIRST_WARPS, lane, s_g);
+        named_barrier_sync(qa::BAR_FIRST, qa::FIRST_WARPS * 32);
+        if (warp == 2)
+            for (int mb = lane; mb < p.qa_first; mb += 32) qa_mark_ready(p, mb);
+        // the rest, a band at a time in order, by warps 2 and 3 while the MMAs run
+        if (warp < 4) {
+            for (int mb0 = p.qa_first; mb0 < p.m_tiles; mb0 += qa::BAND) {
+                const int mb1 = min(mb0 + qa::BAND, p.m_tiles);
+                qa_quantize_range<qa::BG_ITEMS>(p, qp, ql, mb0, mb1, blockIdx.x * qa::BG_WARPS + (warp - 2),
+                                                gridDim.x * qa::BG_WARPS, lane, s_g);
+                named_barrier_sync(qa::BAR_BG, qa::BG_WARPS * 32);
+                if (warp == 2 && mb0 + lane < mb1) qa_mark_ready(p, mb0 + lane);
+            }
+        }
+    }
+
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int t = tile + p.tile_shift - (tile + p.tile_shift >= num_tiles ? num_tiles : 0);
-                const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+        // (the whole warp walks the tiles, for the ready check of QA; lane 0
+        // issues the copies)
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int ready_below = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int t = tile + p.tile_shift - (tile + p.tile_shift >= num_tiles ? num_tiles : 0);
+            int mb, nb;
+            tile_mn<QA>(t, p, mb, nb);
+            if (QA && mb >= ready_below) ok = qa_wait_ready(p, ready_below, mb, lane);
+            if (lane == 0 && ok) {
                 for (int kt = 0; kt < p.k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, kStatusTimeoutEmpty)) {
                         ok = false;
@@ -275,12 +438,13 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                     }
                 }
             }
-            if (!ok) {
-                // Give the copies already issued a bounded time to land before the
-                // CTA can leave (they need nothing else to complete).
-                const long long t0 = clock64();
-                while (clock64() - t0 < kWaitCycles / 64) {
-                }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (lane == 0 && !ok) {
+            // Give the copies already issued a bounded time to land before the
+            // CTA can leave (they need nothing else to complete).
+            const long long t0 = clock64();
+            while (clock64() - t0 < kWaitCycles / 64) {
             }
         }
         __syncwarp();
@@ -417,7 +581,8 @@ __global__ void __launch_bounds__(large::THREADS, 1)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int b = i & 1;
             const int t = tile + p.tile_shift - (tile + p.tile_shift >= num_tiles ? num_tiles : 0);
-            const int mb = t % p.m_tiles, nb = t / p.m_tiles;
+            int mb, nb;
+            tile_mn<QA>(t, p, mb, nb);
             if (!mbar_wait(&acc_full[b], (i >> 1) & 1, kStatusTimeoutAccum)) break;
             tc_fence_after();
             const int row = mb * BM + quad * 32 + lane;

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <mutex>
@@ -83,6 +84,8 @@ nvfp4_status device_state(DeviceState** out)
                                             large::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             large::SMEM_BYTES));
+        NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_large_kernel<false, true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, large::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             pairk::SMEM_BYTES));
         NVFP4_CUDA_TRY(cudaFuncSetAttribute(gemm_decode_kernel<16, false>,
@@ -341,6 +344,16 @@ unsigned long long next_epoch()
     return g_epoch.fetch_add(2ull) + 2ull;
 }
 
+// Per-call tags of the fused prefill kernel's ready words: 1, 2, 3, ... in
+// this process (the kernel raises each word to the current tag with an atomic
+// maximum, so tags must grow; 2^32 - 1 calls before they wrap).
+std::atomic<unsigned int> g_prefill_tag{0};
+
+unsigned long long next_prefill_tag()
+{
+    return (unsigned long long)g_prefill_tag.fetch_add(1u) + 1ull;
+}
+
 template <int BT, bool FQ>
 nvfp4_status launch_decode(const DecodeMaps& maps, const GemmParams& p, cudaStream_t s)
 {
@@ -424,6 +437,23 @@ size_t nvfp4_gemm_workspace_size(int64_t m, int64_t n, int64_t k, uint32_t flags
     (void)k;
     const bool decode_path = flags == NVFP4_GEMM_FORCE_DECODE || (flags == NVFP4_GEMM_AUTO && m <= 64);
     return decode_path && m >= 0 && m <= 64 ? decode_ws_bytes(m) : 0;
+}
+
+int nvfp4_gemm_kernel_for(int64_t m, int64_t n, int sms, uint32_t flags, int with_gates)
+{
+    if (m < 0 || n <= 0 || sms <= 0 || flags > NVFP4_GEMM_FORCE_LARGE_PAIR) return -1;
+    if (flags != NVFP4_GEMM_AUTO) return (int)flags;
+    if (m <= 64) return (int)NVFP4_GEMM_FORCE_DECODE;
+    // Large M: the CTA-pair kernel (256 x 256 tiles on two SMs) when it needs
+    // no more waves of tiles than the single-CTA kernel (128 x 256 tiles, one
+    // per SM).  Per SM the two do the same work per wave and the pair kernel
+    // runs each wave about 2 % faster.  Calls with gate outputs keep the
+    // single-CTA kernel, which schedules the gate tiles first.
+    if (with_gates || m < 256 || sms < 2) return (int)NVFP4_GEMM_FORCE_LARGE;
+    const int64_t n_blocks = (n + 255) / 256;
+    const int64_t single_waves = ((m + 127) / 128 * n_blocks + sms - 1) / sms;
+    const int64_t pair_waves = ((m + 255) / 256 * n_blocks + sms / 2 - 1) / (sms / 2);
+    return (int)(pair_waves <= single_waves ? NVFP4_GEMM_FORCE_LARGE_PAIR : NVFP4_GEMM_FORCE_LARGE);
 }
 
 const char* nvfp4_get_last_error_string(void) { return g_err; }
@@ -665,8 +695,10 @@ static nvfp4_status gemm_impl(const uint8_t* a_q, const uint8_t* a_sf, const flo
         p.gdn_ld = gates->ldg;
     }
 
+    const bool use_pair =
+        !use_decode && nvfp4_gemm_kernel_for(m, n, dev->sms, flags, gates != nullptr) == (int)NVFP4_GEMM_FORCE_LARGE_PAIR;
     CUtensorMap ta, tw;
-    if (!use_decode && flags != NVFP4_GEMM_FORCE_LARGE_PAIR) {
+    if (!use_decode && !use_pair) {
         p.m_tiles = (int)((m + large::BM - 1) / large::BM);
         p.n_tiles = (int)((n + large::BN - 1) / large::BN);
         if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
@@ -892,6 +924,94 @@ nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int64_t m, in
     else if (bt == 32) st = launch_decode<32, true>(maps, p, s);
     else st = launch_decode<64, true>(maps, p, s);
     if (st != NVFP4_OK) return st;
+    return ok();
+}
+
+size_t nvfp4_linear_prefill_workspace_size(int64_t m)
+{
+    if (m < 0) return 0;
+    return (size_t)pad_to((m + 127) / 128 * 8, 16);
+}
+
+nvfp4_status nvfp4_linear_prefill(const void* a, nvfp4_in_dtype dt, int64_t m, int64_t k, int64_t lda,
+                                  const float* act_scale_dev, uint8_t* a_q, uint8_t* a_sf, const uint8_t* w_q,
+                                  const uint8_t* w_sf, int64_t n, const nvfp4_segment* segs, int nsegs, void* c,
+                                  nvfp4_out_dtype odt, int64_t ldc, void* workspace, size_t ws_bytes, void* stream)
+{
+    nvfp4_status st = check_quant_input(a, dt, m, k, lda, "linear_prefill");
+    if (st != NVFP4_OK) return st;
+    if (dt != NVFP4_IN_BF16)
+        return fail(NVFP4_ERR_UNSUPPORTED, "linear_prefill: BF16 activations only (use nvfp4_quantize_act + nvfp4_gemm)");
+    if (m > 0 && m <= 64)
+        return fail(NVFP4_ERR_UNSUPPORTED, "linear_prefill: m = %lld <= 64 (use nvfp4_linear_decode)", (long long)m);
+    if (act_scale_dev == nullptr)
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_prefill: needs the static activation scale act_scale_dev");
+    if (n <= 0 || n % 16 != 0)
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_prefill: n must be a positive multiple of 16 (n=%lld)", (long long)n);
+    if (n >= (1ll << 31)) return fail(NVFP4_ERR_UNSUPPORTED, "linear_prefill: dimension >= 2^31");
+    if (odt != NVFP4_OUT_BF16 && odt != NVFP4_OUT_FP32)
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_prefill: bad output dtype");
+    if (ldc < n) return fail(NVFP4_ERR_INVALID_ARG, "linear_prefill: ldc %lld < n %lld", (long long)ldc, (long long)n);
+    SegTable table;
+    if ((st = check_segments(segs, nsegs, n, &table)) != NVFP4_OK) return st;
+    if (m > 0 && (a_q == nullptr || a_sf == nullptr || w_q == nullptr || w_sf == nullptr || c == nullptr))
+        return fail(NVFP4_ERR_INVALID_ARG, "linear_prefill: NULL pointer");
+    const int64_t osz = odt == NVFP4_OUT_FP32 ? 4 : 2;
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(c) ||
+        (ldc * osz) % 16 != 0)
+        return fail(NVFP4_ERR_ALIGNMENT, "linear_prefill: buffers and output rows must be 16-byte aligned");
+    if (workspace == nullptr || ws_bytes < nvfp4_linear_prefill_workspace_size(m))
+        return fail(NVFP4_ERR_WORKSPACE, "linear_prefill: needs %zu bytes of workspace (got %zu)",
+                    nvfp4_linear_prefill_workspace_size(m), ws_bytes);
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "linear_prefill: workspace not 16-byte aligned");
+    if (m == 0) return ok();
+
+    DeviceState* dev = nullptr;
+    if ((st = device_state(&dev)) != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GemmParams p = {};
+    p.m = (int)m;
+    p.n = (int)n;
+    p.k = (int)k;
+    p.a_sf = a_sf;
+    p.w_sf = w_sf;
+    p.act_scale = act_scale_dev;
+    p.c = c;
+    p.ldc = ldc;
+    p.out_fp32 = odt == NVFP4_OUT_FP32;
+    p.segs = table;
+    p.katoms = (int)(pad_to(k / 16, 4) / 4);
+    p.k_tiles = (int)((k + 255) / 256);
+    p.a_rowblocks = (int)((m + 127) / 128);
+    p.w_rowblocks = (int)((n + 127) / 128);
+    p.splits = 1;
+    p.a_in = a;
+    p.lda = lda;
+    p.qa_q = a_q;
+    p.qa_sf = a_sf;
+    p.qa_ready = static_cast<unsigned long long*>(workspace);
+    p.epoch = next_prefill_tag();
+    p.m_tiles = (int)((m + large::BM - 1) / large::BM);
+    p.n_tiles = (int)((n + large::BN - 1) / large::BN);
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    const int grid = (int)(tiles < dev->sms ? tiles : dev->sms);
+    // m-blocks quantised before the mainloop: those the first two waves of
+    // tiles read (band b of the tile order holds m-blocks [BAND b, BAND b +
+    // BAND), column-major inside the band)
+    {
+        const int64_t last = std::min<int64_t>(tiles, 2 * (int64_t)grid) - 1;
+        const int64_t band_tiles = (int64_t)qa::BAND * p.n_tiles;
+        const int64_t band = last / band_tiles;
+        const int64_t r = last - band * band_tiles;
+        const int64_t bsz = std::min<int64_t>(qa::BAND, p.m_tiles - band * qa::BAND);
+        p.qa_first = (int)(band * qa::BAND + std::min<int64_t>(r + 1, bsz));
+    }
+    CUtensorMap ta, tw, tc;
+    if ((st = encode_fp4_map(&ta, a_q, m, k, large::BM)) != NVFP4_OK) return st;
+    if ((st = encode_fp4_map(&tw, w_q, n, k, large::BN)) != NVFP4_OK) return st;
+    if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
+    gemm_large_kernel<false, true><<<grid, large::THREADS, large::SMEM_BYTES, s>>>(ta, tw, tc, p);
+    NVFP4_CUDA_TRY(cudaGetLastError());
     return ok();
 }
 

@@ -21,6 +21,7 @@ enum : uint32_t {
     kStatusTimeoutCluster = 1u << 3,   // decode: another CTA's partial tile never published
     kStatusTimeoutSelftest = 1u << 4,  // the deliberate self-test wait
     kStatusTimeoutDrain = 1u << 5,     // waiting for in-flight copies after an abort
+    kStatusTimeoutQuant = 1u << 6,     // large M with fused quantisation: rows of A never became ready
 };
 
 __device__ unsigned int g_device_status;
@@ -162,6 +163,26 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes)
 __device__ __forceinline__ void fence_proxy_async_shared()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The same for global memory: generic stores that TMA loads (the async
+// proxy) of other CTAs read after a release/acquire hand-off.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_volatile_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Named barrier `id` (1..15) over `threads` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // ---------------------------------------------------------------------------

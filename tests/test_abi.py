@@ -284,3 +284,40 @@ def test_new_bindings_refuse_host_tensors(lib):
         nv.kv_cache_quantize_fp8(x, x, one, one, cache, cache.clone())
     with pytest.raises(ValueError, match="CUDA"):
         nv.gemm_gdn(None, None, 0, 48, torch.zeros(48), torch.zeros(48))
+
+
+def test_gemm_kernel_choice(lib):
+    """AUTO: decode kernel up to 64 tokens; above, the CTA-pair kernel where it
+    needs no more waves of tiles than the single-CTA kernel (148 SMs)."""
+    import nvfp4_w4a4_quantized_07_b200 as nv
+    pick = nv.gemm_kernel_for
+    D, L, P = nv.NVFP4_GEMM_FORCE_DECODE, nv.NVFP4_GEMM_FORCE_LARGE, nv.NVFP4_GEMM_FORCE_LARGE_PAIR
+    assert pick(1, 5120, 148) == D and pick(64, 34816, 148) == D
+    assert pick(65, 5120, 148) == L and pick(255, 5120, 148) == L
+    # 8192 x 12384: 64 x 49 = 3136 tiles = 22 waves; pairs: 32 x 49 = 1568 on 74 pairs = 22 waves
+    assert pick(8192, 12384, 148) == P
+    assert pick(4096, 5120, 148) == P                  # 5 waves either way
+    assert pick(3712, 5120, 148) == L                  # 4 waves against 5 (29 row tiles do not pair up)
+    assert pick(4736, 5120, 148) == L                  # 740 tiles = 5 waves; 380 pair tiles = 6 waves
+    assert pick(8192, 12384, 148, with_gates=True) == L
+    assert pick(8192, 12384, 148, flags=L) == L and pick(8, 128, 148, flags=P) == P
+    assert pick(-1, 16, 148) == -1 and pick(16, 16, 0) == -1 and pick(16, 16, 148, flags=9) == -1
+
+
+def test_linear_prefill_argument_errors(lib):
+    f = lib.nvfp4_linear_prefill
+    s = _segs((0, 256, 1.0))
+    ws = ctypes.c_void_p(0x40000)
+    need = lib.nvfp4_linear_prefill_workspace_size(300)
+    assert need == 16 * ((3 * 8 + 15) // 16) and lib.nvfp4_linear_prefill_workspace_size(-1) == 0
+    args = lambda m=300, dt=0, k=256, scale=FAKE, a=FAKE, wsp=ws, wsb=need, segs=s, n=256: (
+        a, dt, m, k, k, scale, FAKE, FAKE, FAKE, FAKE, n, segs, 1, FAKE, 0, n, wsp, wsb, None)
+    assert f(*args(m=64)) == 2                        # m <= 64: the decode layer's job
+    assert f(*args(dt=1)) == 2                        # FP32 activations: two-call path
+    assert f(*args(scale=None)) == 1                  # static scale required
+    assert f(*args(k=48)) == 1                        # k % 32
+    assert f(*args(wsp=None, wsb=0)) == 6             # workspace
+    assert f(*args(wsb=need - 16)) == 6
+    assert f(*args(a=MISALIGNED)) == 3
+    assert f(*args(segs=_segs((0, 128, 1.0)))) == 1   # segments do not cover n
+    assert f(*args(m=0)) == 0                         # empty

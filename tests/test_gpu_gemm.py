@@ -197,7 +197,7 @@ def test_config_prefill_4096x5120x5120_sampled_rows():
     assert torch.equal(c.cpu(), c32.cpu().to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("flags", [AUTO, PAIR])
+@pytest.mark.parametrize("flags", [AUTO, LARGE, PAIR])
 def test_config_fused_gdn_in_proj_8192_sampled_rows(flags):
     """8192 x 5120 activations against six separately calibrated modules
     [2048, 2048, 4096, 4096, 48, 48] (N = 12384), checked against the oracle
