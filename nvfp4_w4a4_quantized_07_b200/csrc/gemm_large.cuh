@@ -772,7 +772,7 @@ constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_C = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int C_WARP = 1024;
+constexpr int C_WARP = 2048;                        // per epilogue warp: one 32 x 32 BF16 chunk
 constexpr int OFF_BAR = OFF_C + 8 * C_WARP;
 constexpr int SF_SLOTS = 2;
 // full[S], empty[S], sf_ready[SLOTS], acc_full[2], acc_empty[2], ovl_free, drain
@@ -1028,26 +1028,22 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[b]), 0));
                 uint8_t* cbuf = smem + OFF_C + ew * C_WARP;
+// One 32 x 32 BF16 chunk per TMA store (this kernel has the shared
+                // memory for a 2 KB buffer per warp; half as many stores as
+                // 16-row chunks, which measured ~1.5 % faster).
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
 #pragma unroll
-                    for (int hr = 0; hr < 2; ++hr) {
-                        if (lane == 0) bulk_wait_group_read<0>();
-                        __syncwarp();
-                        if ((lane >> 4) == hr) {
-                            const int r = lane & 15;
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                *reinterpret_cast<uint4*>(cbuf + r * 64 + ((u ^ ((r >> 1) & 3)) << 4)) =
-                                    make_uint4(packed[j][4 * u], packed[j][4 * u + 1], packed[j][4 * u + 2],
-                                               packed[j][4 * u + 3]);
-                        }
-                        fence_proxy_async_shared();
-                        __syncwarp();
-                        if (lane == 0 && row0 + 16 * hr < p.m && ncol0 + j * 32 < p.n) {
-                            tma_store_2d(&tmap_c, cbuf, ncol0 + j * 32, row0 + 16 * hr);
-                            bulk_commit_group();
-                        }
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<uint4*>(cbuf + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(packed[j][4 * u], packed[j][4 * u + 1], packed[j][4 * u + 2], packed[j][4 * u + 3]);
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0 && row0 < p.m && ncol0 + j * 32 < p.n) {
+                        tma_store_2d(&tmap_c, cbuf, ncol0 + j * 32, row0);
+                        bulk_commit_group();
                     }
                 }
                 if (gdn_touches(p, ncol0, 128)) gdn_pass(p, cbuf, packed, row0, ncol0, lane);

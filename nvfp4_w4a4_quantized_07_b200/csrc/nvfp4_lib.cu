@@ -184,11 +184,13 @@ nvfp4_status encode_decode_maps(DecodeMaps* m, const uint8_t* a_q, const uint8_t
 // (64-byte swizzle); the FP32 map (32 x 32, 128-byte swizzle) is encoded for
 // completeness, FP32 output is written with plain stores.  Stores past m or n
 // are clipped by the copy engine.
-nvfp4_status encode_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64_t ldc, bool fp32)
+// Output map: boxes of 32 columns x `bf16_rows` rows (BF16, 64-byte swizzle)
+// or 32 x 32 (FP32, 128-byte swizzle).
+nvfp4_status encode_c_map(CUtensorMap* map, void* c, int64_t m, int64_t n, int64_t ldc, bool fp32, int bf16_rows = 16)
 {
     const cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)m};
     const cuuint64_t strides[1] = {(cuuint64_t)(ldc * (fp32 ? 4 : 2))};
-    const cuuint32_t box[2] = {32u, fp32 ? 32u : 16u};
+    const cuuint32_t box[2] = {32u, fp32 ? 32u : (cuuint32_t)bf16_rows};
     const cuuint32_t estr[2] = {1u, 1u};
     CUresult r = g_encode(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -729,7 +731,7 @@ static nvfp4_status gemm_impl(const uint8_t* a_q, const uint8_t* a_sf, const flo
         if ((st = encode_fp4_map(&ta, a_q, m, k, pairk::CTA_ROWS)) != NVFP4_OK) return st;
         if ((st = encode_fp4_map(&tw, w_q, n, k, pairk::BN / 2)) != NVFP4_OK) return st;
         CUtensorMap tc;
-        if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0)) != NVFP4_OK) return st;
+        if ((st = encode_c_map(&tc, c, m, n, ldc, p.out_fp32 != 0, 32)) != NVFP4_OK) return st;
         const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
         const int pairs = (int)(tiles < dev->sms / 2 ? tiles : dev->sms / 2);
         cudaLaunchConfig_t cfg = {};
