@@ -1028,7 +1028,7 @@ __global__ void __launch_bounds__(pairk::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_remote(map_shared_rank(smem_u32(&acc_empty[b]), 0));
                 uint8_t* cbuf = smem + OFF_C + ew * C_WARP;
-// One 32 x 32 BF16 chunk per TMA store (this kernel has the shared
+                // One 32 x 32 BF16 chunk per TMA store (this kernel has the shared
                 // memory for a 2 KB buffer per warp; half as many stores as
                 // 16-row chunks, which measured ~1.5 % faster).
 #pragma unroll
