@@ -260,14 +260,12 @@ NVFP4_API nvfp4_status nvfp4_gemm_gdn(const uint8_t* a_q, const uint8_t* a_sf, c
  * with the same static scale.  The pages do not describe the MLP; this is the
  * step between its two W4A4 linear layers.
  *
- * Performance: on B200 this call is SLOWER than the two-call path it
- * replaces, although it writes a ninth of the bytes.  Measured at m = 8192,
- * f = 17408, k = 5120: 0.95 ms, against 0.63 ms for nvfp4_gemm (BF16 out)
- * plus about 0.25 ms for nvfp4_silu_mul_quantize.  The per-element silu,
- * division and block quantisation in the epilogue take longer than the next
- * tile's MMAs, so the epilogue sets the pace (tensor pipe busy 37 % of the
- * time against 59 %).  Use it where the m x 2f BF16 intermediate cannot be
- * afforded; otherwise prefer the two calls.
+ * Performance: on B200 this call is faster than the two-call path it
+ * replaces and writes a ninth of the bytes.  Measured at m = 8192,
+ * f = 17408, k = 5120: 0.62 ms, against 0.59 ms for nvfp4_gemm (BF16 out)
+ * plus 0.25-0.26 ms for nvfp4_silu_mul_quantize.  (It was slower, 0.95 ms,
+ * while its epilogue released the accumulator columns the next tile shares
+ * only after the SiLU arithmetic; it now releases them first.)
  *
  *   a_q, a_sf, act_scale_dev  quantised activations, m x k (as for nvfp4_gemm).
  *   w_q, w_sf                 fused weight, 2f rows; f a multiple of 128.

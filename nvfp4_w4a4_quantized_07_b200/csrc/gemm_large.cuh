@@ -328,6 +328,59 @@ __device__ __forceinline__ bool qa_wait_ready(const GemmParams& p, int& ready_be
     return true;
 }
 
+// SwiGLU epilogue, first half: the warp's two gate chunks and two up chunks
+// (items 0, 1: gate g2 = 0, 1 = chunks 2 HALF + g2; items 2, 3: up = those + 4)
+// as the BF16 values the unfused GEMM would store, packed in pairs.  The
+// chunks the other accumulator shares (ACC0: chunk >= 5, ACC1: chunk <= 2)
+// are loaded first, together, and released before anything else, so the next
+// tile's MMAs do not wait for this warp's arithmetic; then the rest, one at a
+// time, and the accumulator is released.
+template <int B, int HALF, typename Release, typename Done>
+__device__ __forceinline__ void swiglu_load(uint32_t tacc, int hcol0, float s_ga, const GemmParams& p, int lane,
+                                            Release release, Done done, uint32_t (&gp)[2][16], uint32_t (&up)[2][16])
+{
+    auto chunk = [](int it) { return 2 * HALF + (it & 1) + (it >= 2 ? 4 : 0); };
+    auto shared = [&](int it) { return B ? chunk(it) <= 2 : chunk(it) >= 5; };
+    auto to_bf16 = [&](const uint32_t (&v)[32], int it, uint32_t (&o)[16]) {
+        const int col = (it >= 2 ? p.swiglu_f : 0) + hcol0 + 32 * (it & 1);
+        const float a0 = __fmul_rn(s_ga, segment_scale(p.segs, col));
+        const float a1 = __fmul_rn(s_ga, segment_scale(p.segs, col + 16));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            o[e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * e]), a0), __fmul_rn(__uint_as_float(v[2 * e + 1]), a0));
+            o[8 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(v[16 + 2 * e]), a1),
+                                   __fmul_rn(__uint_as_float(v[16 + 2 * e + 1]), a1));
+        }
+    };
+    auto dst = [&](int it) -> uint32_t(&)[16] { return it >= 2 ? up[it & 1] : gp[it & 1]; };
+    // the shared items (one or two; every warp holds at least one)
+    constexpr int S0 = (B ? (2 * HALF + 0 <= 2) : false) ? 0 : (B ? (2 * HALF + 1 <= 2 ? 1 : -1) : (2 * HALF + 4 >= 5 ? 2 : 3));
+    static_assert(S0 >= 0, "every epilogue warp holds a shared chunk");
+    constexpr int S1 = B ? ((S0 == 0 && 2 * HALF + 1 <= 2) ? 1 : -1) : ((S0 == 2) ? 3 : -1);
+    {
+        uint32_t va[32], vb[32];
+        tmem_ld_32x32b_x32(tacc + chunk(S0) * 32, va);
+        if constexpr (S1 >= 0) tmem_ld_32x32b_x32(tacc + chunk(S1) * 32, vb);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) release();
+        to_bf16(va, S0, dst(S0));
+        if constexpr (S1 >= 0) to_bf16(vb, S1, dst(S1));
+    }
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        if (it == S0 || it == S1) continue;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tacc + chunk(it) * 32, v);
+        tmem_ld_wait();
+        to_bf16(v, it, dst(it));
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) done();
+}
+
 // SWIGLU: the gate/up GEMM of a gated MLP with its glue fused into the
 // epilogue.  Each 128 x 256 tile holds 128 gate columns (accumulator columns
 // 0..127) and the matching 128 up columns (128..255), loaded as two 128-row
@@ -616,36 +669,44 @@ __global__ void __launch_bounds__(large::THREADS, 1)
             const int ov_rot = OV::rot(b, half), ov_count = OV::count(b, half);
             if (SWIGLU) {
                 // warp (quad, half): gate chunks 2 half, 2 half + 1 with the up
-                // chunks 4 columns-of-32 to the right; 64 h columns per row
+                // chunks 4 columns-of-32 to the right; 64 h columns per row.
+                // Each chunk is first turned into the BF16 values the unfused
+                // GEMM would store (g, u); the chunks the other accumulator
+                // shares are loaded first and released before the rest (chunk
+                // c of ACC0 is shared when c >= 5, of ACC1 when c <= 2), so the
+                // next tile's MMAs do not wait for the SiLU arithmetic.
                 const uint32_t tacc = tmem_base + ((uint32_t)(quad * 32) << 16) + (b ? ACC1_COL : 0);
                 const float s_h = *p.h_scale;
                 const int hcol0 = nb * 128 + half * 64;             // first h column of this warp
+                uint32_t gpk[2][16], upk[2][16];                    // BF16 pairs of g and u
+                auto rel = [&] { mbar_arrive(ovl_free); };
+                auto done = [&] { mbar_arrive(&acc_empty[b]); };
+                if (b == 0) {
+                    if (half == 0) swiglu_load<0, 0>(tacc, hcol0, s_ga, p, lane, rel, done, gpk, upk);
+                    else swiglu_load<0, 1>(tacc, hcol0, s_ga, p, lane, rel, done, gpk, upk);
+                } else {
+                    if (half == 0) swiglu_load<1, 0>(tacc, hcol0, s_ga, p, lane, rel, done, gpk, upk);
+                    else swiglu_load<1, 1>(tacc, hcol0, s_ga, p, lane, rel, done, gpk, upk);
+                }
                 uint32_t sfw = 0;
+                const bool live = row < p.m;
 #pragma unroll
                 for (int g2 = 0; g2 < 2; ++g2) {
-                    const int gc = 2 * half + g2;                    // gate chunk; up chunk is gc + 4
-                    uint32_t vg[32], vu[32];
-                    tmem_ld_32x32b_x32(tacc + gc * 32, vg);
-                    tmem_ld_32x32b_x32(tacc + (gc + 4) * 32, vu);
-                    tmem_ld_wait();
                     const int gcol = hcol0 + 32 * g2;                // gate column in the fused weight
-                    const float ag0 = __fmul_rn(s_ga, segment_scale(p.segs, gcol));
-                    const float ag1 = __fmul_rn(s_ga, segment_scale(p.segs, gcol + 16));
-                    const float au0 = __fmul_rn(s_ga, segment_scale(p.segs, p.swiglu_f + gcol));
-                    const float au1 = __fmul_rn(s_ga, segment_scale(p.segs, p.swiglu_f + gcol + 16));
+                    const uint32_t(&gp)[16] = gpk[g2];
+                    const uint32_t(&up)[16] = upk[g2];
                     float h0[16], h1[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float g0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vg[e]), ag0)));
-                        const float u0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vu[e]), au0)));
-                        const float g1 =
-                            __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vg[16 + e]), ag1)));
-                        const float u1 =
-                            __bfloat162float(__float2bfloat16_rn(__fmul_rn(__uint_as_float(vu[16 + e]), au1)));
-                        h0[e] = silu_mul_bf16(g0, u0);
-                        h1[e] = silu_mul_bf16(g1, u1);
+                    for (int e = 0; e < 8; ++e) {
+                        const float g0l = __uint_as_float(gp[e] << 16), g0h = __uint_as_float(gp[e] & 0xFFFF0000u);
+                        const float u0l = __uint_as_float(up[e] << 16), u0h = __uint_as_float(up[e] & 0xFFFF0000u);
+                        const float g1l = __uint_as_float(gp[8 + e] << 16), g1h = __uint_as_float(gp[8 + e] & 0xFFFF0000u);
+                        const float u1l = __uint_as_float(up[8 + e] << 16), u1h = __uint_as_float(up[8 + e] & 0xFFFF0000u);
+                        h0[2 * e] = silu_mul_bf16(g0l, u0l);
+                        h0[2 * e + 1] = silu_mul_bf16(g0h, u0h);
+                        h1[2 * e] = silu_mul_bf16(g1l, u1l);
+                        h1[2 * e + 1] = silu_mul_bf16(g1h, u1h);
                     }
-                    const bool live = row < p.m;
                     uint32_t sb0, sb1;
                     uint2 q0, q1;
                     quantize_block16(h0, s_h, live, sb0, q0);
@@ -654,12 +715,6 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                         *reinterpret_cast<uint4*>(p.h_q + (int64_t)row * (p.swiglu_f >> 1) + (gcol >> 1)) =
                             make_uint4(q0.x, q0.y, q1.x, q1.y);
                     sfw |= (sb0 | (sb1 << 8)) << (16 * g2);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(ovl_free);
-                    mbar_arrive(&acc_empty[b]);
                 }
                 // four consecutive 16-column blocks of h: one word of the row's atom
                 // (zero on the padding rows, which the tiled layout requires)
