@@ -168,6 +168,66 @@ __device__ __forceinline__ void gdn_pass(const GemmParams& p, uint8_t* cbuf, con
     }
 }
 
+// Stage unit (chunk j, row half hr) of `packed` into a 16 x 32 buffer: the
+// 16 lanes of that half each write their row.
+__device__ __forceinline__ void stage_unit(uint8_t* buf, const uint32_t (&packed)[4][16], int j, int hr, int lane)
+{
+    if ((lane >> 4) != hr) return;
+    const int r = lane & 15;
+    switch (j) {
+        case 0: stage_chunk_row<0>(buf, packed, r); break;
+        case 1: stage_chunk_row<1>(buf, packed, r); break;
+        case 2: stage_chunk_row<2>(buf, packed, r); break;
+        default: stage_chunk_row<3>(buf, packed, r); break;
+    }
+}
+
+// The gate pass when only one half of a tile (owner_half) holds gate columns:
+// the two epilogue warps of the quadrant share it.  The owner holds the
+// values; unit by unit (16 rows x 32 columns) it stages one unit into its
+// own 1 KB buffer and the next into its partner's, and each warp computes the
+// gates of the unit in its buffer (named barrier 10 + quad between the two
+// warps).  In the fused GDN in-proj the gate columns all fall in one half of
+// the last tile column, whose other half lies past N, so this halves the gate
+// work per warp.
+__device__ __forceinline__ void gdn_pass_shared(const GemmParams& p, uint8_t* cbase, int c_warp,
+                                                const uint32_t (&packed)[4][16], int row0, int nb0, int quad,
+                                                int half, int owner_half, int lane)
+{
+    uint8_t* own_buf = cbase + (owner_half * 4 + quad) * c_warp;
+    uint8_t* help_buf = cbase + ((1 - owner_half) * 4 + quad) * c_warp;
+    const int ncol0 = nb0 + owner_half * 128;
+    const bool is_owner = half == owner_half;
+    const int bar = 10 + quad;
+    if (lane == 0) bulk_wait_group_read<0>();  // this warp's last TMA store has read its buffer
+    __syncwarp();
+    named_barrier_sync(bar, 64);               // both buffers are free
+    int k = 0, pj = -1, phr = 0;
+#pragma unroll 1
+    for (int q = 0; q < 8; ++q) {
+        const int j = q >> 1, hr = q & 1;
+        if (!gdn_touches(p, ncol0 + j * 32, 32)) continue;
+        if ((k & 1) == 0) {
+            if (is_owner) stage_unit(own_buf, packed, j, hr, lane);
+            pj = j;
+            phr = hr;
+        } else {
+            if (is_owner) stage_unit(help_buf, packed, j, hr, lane);
+            named_barrier_sync(bar, 64);       // staged
+            if (is_owner) gdn_chunk(p, own_buf, row0 + 16 * phr, ncol0 + pj * 32, lane);
+            else gdn_chunk(p, help_buf, row0 + 16 * hr, ncol0 + j * 32, lane);
+            named_barrier_sync(bar, 64);       // read: the buffers may be restaged
+            pj = -1;
+        }
+        ++k;
+    }
+    if (pj >= 0) {
+        named_barrier_sync(bar, 64);
+        if (is_owner) gdn_chunk(p, own_buf, row0 + 16 * phr, ncol0 + pj * 32, lane);
+        named_barrier_sync(bar, 64);
+    }
+}
+
 namespace large {
 constexpr int BM = 128, BN = 256, BK_BYTES = 128;  // BK = 256 FP4 values per stage
 constexpr int STAGES = 4;
@@ -753,7 +813,16 @@ __global__ void __launch_bounds__(large::THREADS, 1)
                         }
                     }
                 }
-                if (gdn_touches(p, ncol0, 128)) gdn_pass(p, cbuf, packed, row0, ncol0, lane);
+                {
+                    // gates: a warp pass over its own columns, or shared by the
+                    // quadrant's two warps when only one half holds gate columns
+                    const int nb0 = nb * BN;
+                    const bool g0 = gdn_touches(p, nb0, 128), g1 = gdn_touches(p, nb0 + 128, 128);
+                    if (g0 != g1)
+                        gdn_pass_shared(p, smem + OFF_C, C_WARP, packed, row0, nb0, quad, half, g1 ? 1 : 0, lane);
+                    else if (g0)
+                        gdn_pass(p, cbuf, packed, row0, ncol0, lane);
+                }
             } else {
                 for (int jj = 0; jj < 4; ++jj) {
                     const int j = (ov_rot + jj) & 3;
