@@ -14,7 +14,8 @@ namespace nvfp4 {
 // Warp roles (16 warps):
 //   0      TMA producer: A/B tiles and the stage's scale atoms into a 4-stage ring
 //   1      MMA issuer: tcgen05 block-scaled MMAs (M=128, N=256, K=64)
-//   2      owns the TMEM allocation
+//   2      owns the TMEM allocation (with the activation quantisation fused
+//          in, 2..3 quantise A in the background, and 2..15 its first bands)
 //   4..11  epilogue: drain the accumulator, scale by s_ga * s_gw[segment],
 //          convert and store 16 x 32 chunks through shared memory with TMA
 //   12..15 scale staging: read each stage's scale atoms from shared memory and
