@@ -337,9 +337,8 @@ NVFP4_API nvfp4_status nvfp4_linear_decode(const void* a, nvfp4_in_dtype dt, int
  * (nvfp4_check_device_status returns NVFP4_ERR_TIMEOUT).
  *
  * Performance: on B200 this single launch is currently SLOWER than
- * nvfp4_quantize_act followed by nvfp4_gemm: 0.272 ms against 0.259-0.265 ms
- * for 8192 x 5120 x 12384, 0.084 ms against 0.077-0.079 ms for
- * 4096 x 5120 x 5120.  Quantising the first 8-16 m-blocks before the first
+ * nvfp4_quantize_act followed by nvfp4_gemm: 0.261 ms against 0.242 ms for
+ * 8192 x 5120 x 12384, 0.083 ms against 0.075 ms for 4096 x 5120 x 5120.  Quantising the first 8-16 m-blocks before the first
  * MMA costs 6-10 us, the two background warps quantise about 0.5 TB/s (a
  * band of 8 m-blocks per ~20 us, late for the 4096-row case), and the banded
  * tile order and the background traffic slow the mainloop by ~4 %.  Use it
