@@ -86,7 +86,7 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_ACC + BT * ACC_PITCH * 4;
     // full[S], empty[S], sf_ready[SLOTS], sf_free[SLOTS], acc_full[2], acc_empty[2], drain, sga_ready
     static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_SLOTS + 6;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, verdicts, s_ga, amax partials
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;     // TMEM base, wait results, s_ga, amax partials
     static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
     static_assert(A_KT % 1024 == 0, "SW128 operand tiles are 1 KB aligned");
     static_assert(OFF_A + STAGES * A_STAGE - A_KT + 128 * KT_BYTES <= OFF_MISC, "MMA A reads stay in the buffer");
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
     uint64_t* sga_ready = drain + 1;   // FQ: the activation scale is in s_ga_smem
     uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* bad = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);        // a wait ran out
-    volatile int* verdict = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);    // epilogue barrier verdict
+    volatile int* wait_ok = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);    // the epilogue's shared wait result
     volatile float* s_ga_smem = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 12); // FQ: the scale used
     volatile float* amax_part = reinterpret_cast<volatile float*>(smem + C::OFF_MISC + 16); // FQ: [2]
     float* acc_stage = reinterpret_cast<float*>(smem + C::OFF_ACC);
@@ -616,17 +616,17 @@ __global__ void __launch_bounds__(decode::THREADS, 1)
             const bool complete = owner && seg_end == (int64_t)(nb + 1) * k_tiles;
             const int b = seg & 1;
 
-            if (et == 0) *verdict = mbar_wait(&acc_full[b], (seg >> 1) & 1, kStatusTimeoutAccum) ? 1 : 0;
+            if (et == 0) *wait_ok = mbar_wait(&acc_full[b], (seg >> 1) & 1, kStatusTimeoutAccum) ? 1 : 0;
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (!*verdict) {
+            if (!*wait_ok) {
                 if (et == 0) *bad = 1;
                 break;
             }
             if (FQ && seg == 0) {
                 // bounded like every wait; the quantiser set it before its first stage
-                if (et == 0) *verdict = mbar_wait(sga_ready, 0, kStatusTimeoutAccum) ? 1 : 0;
+                if (et == 0) *wait_ok = mbar_wait(sga_ready, 0, kStatusTimeoutAccum) ? 1 : 0;
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (!*verdict) {
+                if (!*wait_ok) {
                     if (et == 0) *bad = 1;
                     break;
                 }
