@@ -152,20 +152,31 @@ def sf_offset(row: int, kblock: int, k: int) -> int:
     return int(load().nvfp4_sf_offset(row, kblock, k))
 
 
+def _ws_key(device):
+    """Cache key of a default workspace: the device and the stream the call
+    runs on (the current stream).  Calls on one stream run in order and may
+    share a workspace; calls on different streams may overlap, so each stream
+    gets its own.  The workspace is allocated while that stream is current, so
+    when a larger one replaces it the caching allocator hands the old memory
+    out again only in that stream's order."""
+    import torch
+    dev = torch.device(device)
+    return dev, int(torch.cuda.current_stream(dev).cuda_stream)
+
+
 _quant_ws_cache = {}
 
 
 def quant_workspace(device) -> "torch.Tensor":
-    """A cached per-device workspace of nvfp4_quant_workspace_size bytes for the
-    dynamic-scale quantisers.  It needs no initialisation (the library clears
-    the amax word it uses on the call's stream), so it is allocated once per
-    device and not filled; calls that may run concurrently on different
-    streams must pass workspaces of their own."""
+    """A cached workspace of nvfp4_quant_workspace_size bytes for the
+    dynamic-scale quantisers, one per (device, current stream).  It needs no
+    initialisation (the library clears the amax word it uses on the call's
+    stream), so it is allocated once and not filled."""
     import torch
-    key = torch.device(device)
+    key = _ws_key(device)
     ws = _quant_ws_cache.get(key)
     if ws is None:
-        ws = torch.empty(load().nvfp4_quant_workspace_size(), dtype=torch.uint8, device=key)
+        ws = torch.empty(load().nvfp4_quant_workspace_size(), dtype=torch.uint8, device=key[0])
         _quant_ws_cache[key] = ws
     return ws
 
@@ -295,16 +306,17 @@ _ws_cache = {}
 
 
 def gemm_workspace(m: int, n: int, k: int, flags: int, device):
-    """A cached per-device workspace of at least nvfp4_gemm_workspace_size bytes
-    (it needs no initialisation: the decode kernel tags what it writes)."""
+    """A cached workspace of at least nvfp4_gemm_workspace_size bytes, one per
+    (device, current stream); it needs no initialisation (the decode kernel
+    tags what it writes)."""
     import torch
     need = int(load().nvfp4_gemm_workspace_size(m, n, k, flags))
     if need == 0:
         return None
-    key = torch.device(device)
+    key = _ws_key(device)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
-        ws = torch.empty(need, dtype=torch.uint8, device=key)
+        ws = torch.empty(need, dtype=torch.uint8, device=key[0])
         _ws_cache[key] = ws
     return ws
 
@@ -504,8 +516,9 @@ def linear_prefill(a, w: FusedWeight, act_scale, out_dtype=None, out=None, a_out
             sf=torch.empty(max(L.nvfp4_sf_bytes(m, k), 1), dtype=torch.uint8, device=a.device),
             scale=act_scale, m=m, k=k)
     if workspace is None:
+        # one per (device, current stream): calls that may overlap must not share it
         need = max(int(L.nvfp4_linear_prefill_workspace_size(m)), 16)
-        key = (a.device.index if a.device.index is not None else torch.cuda.current_device())
+        key = _ws_key(a.device)
         ws = _prefill_ws_cache.get(key)
         if ws is None or ws.numel() < need:
             ws = torch.zeros(need, dtype=torch.uint8, device=a.device)   # zeroed once, as the call requires

@@ -321,3 +321,50 @@ def test_linear_prefill_argument_errors(lib):
     assert f(*args(a=MISALIGNED)) == 3
     assert f(*args(segs=_segs((0, 128, 1.0)))) == 1   # segments do not cover n
     assert f(*args(m=0)) == 0                         # empty
+
+
+def test_default_workspaces_are_per_device_and_stream(lib, monkeypatch):
+    """The binding's default workspaces (dynamic-scale quantisers, decode GEMM
+    partials, one-launch prefill ready words) are cached per (device, current
+    stream): calls on one stream reuse one buffer, calls on another stream get
+    their own, and a larger need replaces the buffer.  Host logic only: the
+    current stream and the device allocations are faked."""
+    import torch
+
+    class FakeStream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    current = {"h": 0x1000}
+    made = []
+    host_empty = torch.empty
+
+    def fake_alloc(*shape, dtype=None, device=None, **kw):
+        assert torch.device(device).type == "cuda"
+        t = host_empty(*shape, dtype=dtype)
+        made.append(t)
+        return t
+
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(current["h"]))
+    monkeypatch.setattr(torch, "empty", fake_alloc)
+    monkeypatch.setattr(nv, "_quant_ws_cache", {})
+    monkeypatch.setattr(nv, "_ws_cache", {})
+
+    q1 = nv.quant_workspace("cuda:0")
+    assert q1.numel() == lib.nvfp4_quant_workspace_size()
+    assert nv.quant_workspace("cuda:0") is q1
+    dec = nv.NVFP4_GEMM_FORCE_DECODE
+    g1 = nv.gemm_workspace(16, 5120, 5120, dec, "cuda:0")
+    assert g1.numel() == lib.nvfp4_gemm_workspace_size(16, 5120, 5120, dec)
+    assert nv.gemm_workspace(1, 5120, 5120, dec, "cuda:0") is g1          # smaller need: same buffer
+    assert nv.gemm_workspace(8192, 5120, 5120, nv.NVFP4_GEMM_AUTO, "cuda:0") is None
+    current["h"] = 0x2000                                                 # another stream
+    q2 = nv.quant_workspace("cuda:0")
+    g2 = nv.gemm_workspace(16, 5120, 5120, dec, "cuda:0")
+    assert q2 is not q1 and g2 is not g1
+    g3 = nv.gemm_workspace(64, 5120, 5120, dec, "cuda:0")                 # larger need: replaced
+    assert g3 is not g2 and g3.numel() == lib.nvfp4_gemm_workspace_size(64, 5120, 5120, dec)
+    current["h"] = 0x1000                                                 # back on the first stream
+    assert nv.quant_workspace("cuda:0") is q1 and nv.gemm_workspace(16, 5120, 5120, dec, "cuda:0") is g1
+    assert nv._ws_key("cuda:0") == (torch.device("cuda:0"), 0x1000)
+    assert len(made) == 5
