@@ -325,7 +325,8 @@ def gemm(a: QuantizedActivation, w: FusedWeight, out_dtype=None, flags: int = NV
          segments=None, out=None, workspace=None):
     """``C = nvfp4_gemm(a, w)``: m x n output, BF16 by default.  ``segments``
     overrides the fused weight's own segment table; ``workspace`` defaults to a
-    cached per-device buffer when the chosen kernel needs one."""
+    buffer cached per (device, current stream) when the chosen kernel needs
+    one."""
     import torch
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     if a.k != w.k:
